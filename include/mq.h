@@ -1,0 +1,177 @@
+/*
+ * mq.h -- C ABI of the nested-bit int8 (Matryoshka Quantization) serving path
+ * for NVIDIA B200 (sm_100a).
+ *
+ * One int8 container per weight matrix serves every width r in {8, 6, 4, 3, 2}:
+ * the r most significant bits are sliced out (Eq. 6), stored as dense r-bit
+ * planes and consumed by a fused unpack -> dequantize -> matmul.
+ * Sources ("Matryoshka Quantization" explainer page): section 3.4 Eq. 1
+ * (MinMax quantizer), "The Bit-Slicing Operator" Eq. 6, section 3.2
+ * ("at deployment, only the int8-quantized model needs to be stored; lower
+ * precisions are extracted by slicing") and "Mix'n'Match and Interpolative
+ * Slicing" (per-layer widths, r = 3 and 6 from the same container).
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, unless a
+ *    comment says otherwise. Every tensor is dense and row-major.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Calls enqueue work on it and return without synchronizing.
+ *  - Arguments are checked on the host before anything is launched. A
+ *    rejected call launches nothing and returns MQ_ERR_INVALID_ARG (bad
+ *    value, null or misaligned pointer) or MQ_ERR_UNSUPPORTED (a valid value
+ *    this build does not serve); mq_last_error() then describes it.
+ *  - A CUDA launch failure returns MQ_ERR_CUDA. A bounded device-side wait
+ *    that gave up is reported by mq_device_status() as MQ_ERR_TIMEOUT.
+ *  - No C++ exception crosses this interface.
+ *  - The library keeps a small per-(device, stream) workspace of device
+ *    memory for its own scratch (activation copies, row sums, error word).
+ *    It is allocated on first use by a call on that stream; make one call
+ *    before capturing such a stream into a CUDA graph. mq_release_workspace()
+ *    frees all of it.
+ */
+#ifndef MQ_H_
+#define MQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MQ_API __attribute__((visibility("default")))
+#else
+#define MQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mq_status {
+  MQ_OK = 0,
+  MQ_ERR_INVALID_ARG = 1,
+  MQ_ERR_UNSUPPORTED = 2,
+  MQ_ERR_CUDA = 3,
+  MQ_ERR_TIMEOUT = 4
+} mq_status;
+
+typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1 } mq_dtype;
+
+/* Library version, (major << 16) | minor. */
+MQ_API int mq_version(void);
+
+/* Text of the last error raised on the calling thread ("" if none). The
+ * pointer stays valid until the next mq_* call on the same thread. */
+MQ_API const char* mq_last_error(void);
+
+/*
+ * Bytes of the dense r-bit planes of an N x K matrix: N*K*r/8.
+ * Returns 0 for N < 1, K < 1, K % 32 != 0 or r not in {8, 6, 4, 3, 2}.
+ * Layout (this library's own; the pages fix only that a slice is an r-bit
+ * integer per weight): r = 8 -> one plane of bytes (the container itself);
+ * r = 4, 2 -> one plane of width r; r = 3 -> planes of widths (2, 1);
+ * r = 6 -> planes of widths (4, 2). Plane 0 holds the low bits of each code,
+ * plane 1 the code shifted right by plane 0's width; the planes follow one
+ * another, each row-major with a row pitch of K*b/8 bytes. In a plane of
+ * width b < 8 every little-endian 32-bit word holds 32/b codes; local code
+ * u sits at bit 16*(u % 2) + b*(u / 2) (even codes in the low half-word, odd
+ * codes in the high half-word). In the byte plane code u sits at bit 8u.
+ */
+MQ_API size_t mq_packed_bytes(int64_t N, int64_t K, int r);
+
+/*
+ * Eq. 1, MinMax asymmetric quantization of each output channel (row) of a
+ * weight matrix into the int8 container:
+ *   alpha_n = (max_k w[n,k] - min_k w[n,k]) / 255,  z_n = -min_k w[n,k] / alpha_n,
+ *   q[n,k]  = clamp(round(w[n,k] / alpha_n + z_n), 0, 255).
+ * Arithmetic contract (IEEE binary32, each operation correctly rounded, no
+ * contraction): d = max - min; alpha = d / 255; z = -min / alpha;
+ * t = (w / alpha) + z; q = clamp(round-half-to-even(t), 0, 255). A row whose
+ * alpha rounds to 0 (max == min) gets alpha = 1 and z = -min (all codes 0).
+ *   w     : N x K, fp32 (dtype MQ_F32) or bf16 (MQ_BF16), 4-byte aligned.
+ *   q     : N x K uint8 out.   alpha, zero : N fp32 out.
+ * Requires N >= 1, K >= 1; weights finite with a finite range.
+ */
+MQ_API mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K,
+                           uint8_t* q, float* alpha, float* zero, void* stream);
+
+/*
+ * Eq. 6 slicing of the container into width r, packed as dense r-bit planes:
+ *   code[n,k] = clamp(round_half_up(q[n,k] / 2^(8-r)), 0, 2^r - 1)
+ * (S(q, r) = code * 2^(8-r); r = 8 is the identity). The first dropped bit
+ * decides the rounding, as the slicing paragraph states.
+ *   q      : N x K uint8 container (from mq_quantize_int8), 16-byte aligned.
+ *   packed : mq_packed_bytes(N, K, r) bytes out, 16-byte aligned.
+ * Requires K % 32 == 0 and r in {8, 6, 4, 3, 2}.
+ */
+MQ_API mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r,
+                        void* packed, void* stream);
+
+/*
+ * Fused unpack -> dequantize -> matmul with a sliced width r:
+ *   y[m,n] = sum_k x[m,k] * alpha_n * (S(q[n,k], r) - z_n)
+ * (dequantization alpha * (q - z) of Eq. 1 with the sliced code in place of
+ * q). x is bf16, accumulation is fp32, y is fp32.
+ *   x      : M x K bf16, 16-byte aligned.
+ *   packed : planes of width r from mq_slice_pack, 16-byte aligned.
+ *   alpha, zero : N fp32 (from mq_quantize_int8).
+ *   y      : M x N fp32 out (overwritten), 4-byte aligned.
+ * Requires 1 <= M, K % 128 == 0 (a 1-bit plane row must be a whole number of
+ * 16-byte units for the bulk copies), N >= 1. M <= 32 runs the decode GEMV
+ * (tensor-core m16n8k16 tiles fed from TMA-staged planes); M > 32 runs the
+ * prefill GEMM (tcgen05, accumulators in tensor memory).
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_k |x[m,k]| |W_r[n,k]| + 1e-6.
+ */
+MQ_API mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed,
+                    const float* alpha, const float* zero, int64_t N, int r,
+                    float* y, void* stream);
+
+/* One linear of a stack: its input, its packed planes, its scales, its output. */
+typedef struct mq_linear_desc {
+  const void* x;       /* M x K bf16 input, 16-byte aligned */
+  const void* packed;  /* planes at the width of the linear's layer */
+  const float* alpha;  /* N */
+  const float* zero;   /* N */
+  float* y;            /* M x N fp32 output (overwritten) */
+  int64_t N;
+  int64_t K;
+} mq_linear_desc;
+
+/*
+ * Mix'n'Match serving: every linear i runs at the width widths[layer_of_lin[i]]
+ * of its layer (the pages' per-layer precision assignment; e.g. int8 on the
+ * outer layers, int2 in the middle). All linears are independent (each reads
+ * its own x), so the whole stack is streamed by one persistent kernel whose
+ * work units run across linear boundaries.
+ *   lins[n_lins], layer_of_lin[n_lins] : HOST arrays.
+ *   widths[n_layers]                  : HOST array, each in {8, 6, 4, 3, 2}.
+ * Requires 1 <= M <= 32 and the mq_linear conditions for every linear.
+ * Stacks longer than 256 linears are split into several launches.
+ */
+MQ_API mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin,
+                           int n_lins, const int* widths, int n_layers,
+                           int64_t M, void* stream);
+
+/*
+ * Synchronizes `stream`, then reports whether any kernel launched by this
+ * library on the current device gave up a bounded wait (MQ_ERR_TIMEOUT; the
+ * outputs of that call are then undefined) and clears the flag.
+ * Returns MQ_ERR_CUDA if the synchronization itself failed.
+ */
+MQ_API mq_status mq_device_status(void* stream);
+
+/* Frees every workspace of this library (all devices and streams). The
+ * caller must ensure no mq_* work is still in flight. */
+MQ_API mq_status mq_release_workspace(void);
+
+/*
+ * Testing hook: the time (ns) a kernel waits on a pipeline barrier before it
+ * gives up, sets the device error flag and exits cleanly. 0 makes every such
+ * wait give up at once (deterministic exercise of the timeout path). The
+ * default is 2 s. Applies to launches made after the call.
+ */
+MQ_API mq_status mq_debug_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MQ_H_ */

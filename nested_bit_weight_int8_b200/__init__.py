@@ -1,0 +1,147 @@
+"""Python binding of libmq.so, the nested-bit int8 (Matryoshka Quantization)
+serving path for B200.
+
+Argument marshalling only: every function forwards to the C ABI declared in
+include/mq.h, and every step of the path runs in the library's CUDA kernels.
+There is no CPU fallback: importing this package fails if libmq.so is missing
+or cannot be loaded.
+
+Pointers are plain integers (device addresses unless documented otherwise);
+helpers accept torch tensors for convenience and pass their data_ptr().
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m nested_bit_weight_int8_b200.build` "
+        "(nvcc, sm_100a). There is no fallback implementation.")
+_lib = ctypes.CDLL(LIB_PATH)
+
+MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CUDA, MQ_ERR_TIMEOUT = range(5)
+MQ_F32, MQ_BF16 = 0, 1
+WIDTHS = (8, 6, 4, 3, 2)
+
+_i64, _int, _vp, _u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64
+
+
+class LinearDesc(ctypes.Structure):
+    """mq_linear_desc: one linear of a Mix'n'Match stack."""
+    _fields_ = [("x", _vp), ("packed", _vp), ("alpha", _vp), ("zero", _vp), ("y", _vp),
+                ("N", _i64), ("K", _i64)]
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_version = _sig("mq_version", _int, [])
+_last_error = _sig("mq_last_error", ctypes.c_char_p, [])
+_packed_bytes = _sig("mq_packed_bytes", ctypes.c_size_t, [_i64, _i64, _int])
+_quantize = _sig("mq_quantize_int8", _int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp])
+_slice_pack = _sig("mq_slice_pack", _int, [_vp, _i64, _i64, _int, _vp, _vp])
+_linear = _sig("mq_linear", _int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
+_stack = _sig("mq_stack_forward", _int,
+              [ctypes.POINTER(LinearDesc), ctypes.POINTER(_int), _int, ctypes.POINTER(_int), _int,
+               _i64, _vp])
+_device_status = _sig("mq_device_status", _int, [_vp])
+_release = _sig("mq_release_workspace", _int, [])
+_wait_limit = _sig("mq_debug_set_wait_limit_ns", _int, [_u64])
+
+EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8",
+            "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
+            "mq_release_workspace", "mq_debug_set_wait_limit_ns")
+
+
+class MQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"mq status {status}: {message}")
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status != MQ_OK:
+        raise MQError(status, _last_error().decode(errors="replace"))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+def version() -> int:
+    return _version()
+
+
+def last_error() -> str:
+    return _last_error().decode(errors="replace")
+
+
+def packed_bytes(N: int, K: int, r: int) -> int:
+    return int(_packed_bytes(N, K, r))
+
+
+def quantize_int8(w, dtype: int, N: int, K: int, q, alpha, zero, stream=None) -> None:
+    """Eq. 1 per-row MinMax int8 container: q (N x K uint8), alpha, zero (N fp32)."""
+    _check(_quantize(_ptr(w), dtype, N, K, _ptr(q), _ptr(alpha), _ptr(zero), _stream(stream)))
+
+
+def slice_pack(q, N: int, K: int, r: int, packed, stream=None) -> None:
+    """Eq. 6 slice of the container at width r, packed as dense r-bit planes."""
+    _check(_slice_pack(_ptr(q), N, K, r, _ptr(packed), _stream(stream)))
+
+
+def linear(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=None) -> None:
+    """y (M x N fp32) = x (M x K bf16) . W_r^T from the packed planes."""
+    _check(_linear(_ptr(x), M, K, _ptr(packed), _ptr(alpha), _ptr(zero), N, r, _ptr(y),
+                   _stream(stream)))
+
+
+def stack_forward(lins, layer_of_lin, widths, M: int, stream=None) -> None:
+    """Mix'n'Match stack. lins: sequence of (x, packed, alpha, zero, y, N, K)."""
+    n = len(lins)
+    arr = (LinearDesc * n)()
+    for i, (x, packed, alpha, zero, y, N, K) in enumerate(lins):
+        arr[i] = LinearDesc(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(zero), _ptr(y), N, K)
+    lol = (_int * n)(*layer_of_lin)
+    wd = (_int * len(widths))(*widths)
+    _check(_stack(arr, lol, n, wd, len(widths), M, _stream(stream)))
+
+
+def device_status(stream=None) -> None:
+    """Synchronizes the stream; raises MQError(MQ_ERR_TIMEOUT) if a kernel gave up a wait."""
+    _check(_device_status(_stream(stream)))
+
+
+def release_workspace() -> None:
+    _check(_release())
+
+
+def debug_set_wait_limit_ns(ns: int) -> None:
+    _check(_wait_limit(ns))
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Calls a C entry point and returns its status code without raising
+    (used by tests of the argument checks)."""
+    return {"mq_quantize_int8": _quantize, "mq_slice_pack": _slice_pack,
+            "mq_linear": _linear}[fn_name](*args)

@@ -1,0 +1,244 @@
+// C ABI entry points: argument checks, status codes, the per-(device, stream)
+// workspace and the device error word. Every compute step runs in the
+// library's own kernels; nothing here computes on the host.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/mq.h"
+#include "mq_internal.h"
+
+namespace mq {
+namespace {
+
+thread_local std::string g_last_error;
+std::mutex g_ws_mutex;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_workspaces;
+std::map<int, uint32_t*> g_error_words;
+uint64_t g_wait_limit_ns = 2000000000ull;
+std::map<int, int> g_sm_counts;
+
+mq_status fail(mq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+mq_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool valid_r(int r) { return r == 8 || r == 6 || r == 4 || r == 3 || r == 2; }
+
+}  // namespace
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_ws_mutex);
+  auto it = g_sm_counts.find(dev);
+  if (it != g_sm_counts.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 1;
+  g_sm_counts[dev] = n;
+  return n;
+}
+
+cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_ws_mutex);
+  Workspace& w = g_workspaces[std::make_pair(dev, stream)];
+  if (w.bytes < bytes) {
+    if (w.ptr) {
+      e = cudaDeviceSynchronize();  // in-flight kernels may still read the old buffer
+      if (e != cudaSuccess) return e;
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    size_t sz = bytes < (1u << 20) ? (1u << 20) : bytes;
+    sz = (sz + 4095) & ~size_t(4095);
+    e = cudaMalloc(&w.ptr, sz);
+    if (e != cudaSuccess) return e;
+    w.bytes = sz;
+  }
+  *out = w.ptr;
+  return cudaSuccess;
+}
+
+cudaError_t get_error_word(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_ws_mutex);
+  auto it = g_error_words.find(dev);
+  if (it == g_error_words.end()) {
+    uint32_t* p = nullptr;
+    e = cudaMalloc(&p, 256);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(p, 0, 256);
+    if (e != cudaSuccess) return e;
+    it = g_error_words.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return cudaSuccess;
+}
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+
+}  // namespace mq
+
+using namespace mq;
+
+extern "C" {
+
+int mq_version(void) { return (0 << 16) | 3; }
+
+const char* mq_last_error(void) { return g_last_error.c_str(); }
+
+size_t mq_packed_bytes(int64_t N, int64_t K, int r) {
+  if (N < 1 || K < 1 || K % 32 != 0 || !valid_r(r)) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) * static_cast<size_t>(r) / 8;
+}
+
+mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
+                           float* alpha, float* zero, void* stream) {
+  g_last_error.clear();
+  if (!w || !q || !alpha || !zero) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: null pointer");
+  if (dtype != MQ_F32 && dtype != MQ_BF16) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: dtype must be MQ_F32 or MQ_BF16");
+  if (N < 1 || K < 1) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: N and K must be >= 1");
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return fail(MQ_ERR_UNSUPPORTED, "mq_quantize_int8: N or K too large");
+  if (!aligned(w, 4) || !aligned(alpha, 4) || !aligned(zero, 4))
+    return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: w, alpha, zero must be 4-byte aligned");
+  cudaError_t e = launch_quantize(w, dtype, N, K, q, alpha, zero, static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "mq_quantize_int8");
+  return MQ_OK;
+}
+
+mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* packed, void* stream) {
+  g_last_error.clear();
+  if (!q || !packed) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: null pointer");
+  if (!valid_r(r)) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: r=%d not in {8,6,4,3,2}", r);
+  if (N < 1 || K < 1 || K % 32 != 0) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: need N >= 1 and K a positive multiple of 32 (K=%lld)", (long long)K);
+  if (!aligned(q, 16) || !aligned(packed, 16)) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: q and packed must be 16-byte aligned");
+  if (N * K > (int64_t(1) << 40)) return fail(MQ_ERR_UNSUPPORTED, "mq_slice_pack: matrix too large");
+  cudaError_t e = launch_slice_pack(q, N, K, r, packed, static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "mq_slice_pack");
+  return MQ_OK;
+}
+
+static mq_status check_linear(const char* who, const void* x, int64_t M, int64_t K, const void* packed,
+                              const float* alpha, const float* zero, int64_t N, int r, const float* y) {
+  if (!x || !packed || !alpha || !zero || !y) return fail(MQ_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!valid_r(r)) return fail(MQ_ERR_INVALID_ARG, "%s: r=%d not in {8,6,4,3,2}", who, r);
+  if (M < 1) return fail(MQ_ERR_INVALID_ARG, "%s: M must be >= 1", who);
+  if (N < 1) return fail(MQ_ERR_INVALID_ARG, "%s: N must be >= 1", who);
+  if (K < 128 || K % 128 != 0) return fail(MQ_ERR_INVALID_ARG, "%s: K must be a positive multiple of 128 (K=%lld)", who, (long long)K);
+  if (!aligned(x, 16) || !aligned(packed, 16)) return fail(MQ_ERR_INVALID_ARG, "%s: x and packed must be 16-byte aligned", who);
+  if (!aligned(alpha, 4) || !aligned(zero, 4) || !aligned(y, 4)) return fail(MQ_ERR_INVALID_ARG, "%s: alpha, zero, y must be 4-byte aligned", who);
+  if (N > (int64_t(1) << 30) || K > (int64_t(1) << 24)) return fail(MQ_ERR_UNSUPPORTED, "%s: N or K too large", who);
+  return MQ_OK;
+}
+
+mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed, const float* alpha,
+                    const float* zero, int64_t N, int r, float* y, void* stream) {
+  g_last_error.clear();
+  mq_status st = check_linear("mq_linear", x, M, K, packed, alpha, zero, N, r, y);
+  if (st != MQ_OK) return st;
+  LinearJob job{x, static_cast<const uint8_t*>(packed), alpha, zero, y, N, K, r};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M <= 32) {
+    e = run_gemv(&job, 1, static_cast<int>(M), s);
+  } else {
+    if (M > (int64_t(1) << 24)) return fail(MQ_ERR_UNSUPPORTED, "mq_linear: M too large");
+    e = run_gemm(job, static_cast<int>(M), s);
+  }
+  if (e == cudaErrorNotSupported) return fail(MQ_ERR_UNSUPPORTED, "mq_linear: shape not served by this build");
+  if (e != cudaSuccess) return cuda_fail(e, "mq_linear");
+  return MQ_OK;
+}
+
+mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, int n_lins,
+                           const int* widths, int n_layers, int64_t M, void* stream) {
+  g_last_error.clear();
+  if (!lins || !layer_of_lin || !widths) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: null host array");
+  if (n_lins < 1 || n_layers < 1) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: need n_lins >= 1 and n_layers >= 1");
+  if (M < 1 || M > 32) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: M must be in [1, 32]");
+  std::vector<LinearJob> jobs(n_lins);
+  for (int i = 0; i < n_lins; ++i) {
+    const int layer = layer_of_lin[i];
+    if (layer < 0 || layer >= n_layers) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: layer_of_lin[%d]=%d out of range", i, layer);
+    const int r = widths[layer];
+    const mq_linear_desc& d = lins[i];
+    char who[64];
+    std::snprintf(who, sizeof(who), "mq_stack_forward[lin %d]", i);
+    mq_status st = check_linear(who, d.x, M, d.K, d.packed, d.alpha, d.zero, d.N, r, d.y);
+    if (st != MQ_OK) return st;
+    jobs[i] = LinearJob{d.x, static_cast<const uint8_t*>(d.packed), d.alpha, d.zero, d.y, d.N, d.K, r};
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int b = 0; b < n_lins; b += kGemvMaxLinears) {
+    const int cnt = (n_lins - b) < kGemvMaxLinears ? (n_lins - b) : kGemvMaxLinears;
+    cudaError_t e = run_gemv(jobs.data() + b, cnt, static_cast<int>(M), s);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_stack_forward");
+  }
+  return MQ_OK;
+}
+
+mq_status mq_device_status(void* stream) {
+  g_last_error.clear();
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+  uint32_t* err = nullptr;
+  e = get_error_word(&err);
+  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+  if (v != 0) {
+    e = cudaMemset(err, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+    return fail(MQ_ERR_TIMEOUT, "a kernel gave up a bounded wait (flags 0x%x); its outputs are undefined", v);
+  }
+  return MQ_OK;
+}
+
+mq_status mq_release_workspace(void) {
+  g_last_error.clear();
+  std::lock_guard<std::mutex> lk(g_ws_mutex);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_workspaces) {
+    if (kv.second.ptr) {
+      cudaSetDevice(kv.first.first);
+      cudaDeviceSynchronize();
+      cudaFree(kv.second.ptr);
+    }
+  }
+  g_workspaces.clear();
+  cudaSetDevice(cur);
+  return MQ_OK;
+}
+
+mq_status mq_debug_set_wait_limit_ns(uint64_t ns) {
+  g_last_error.clear();
+  g_wait_limit_ns = ns;
+  return MQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+namespace mq {
+
+// One sliced linear as the host planner sees it (device pointers).
+struct LinearJob {
+  const void* x;        // M x K bf16
+  const uint8_t* packed;
+  const float* alpha;
+  const float* zero;
+  float* y;             // M x N fp32
+  int64_t N;
+  int64_t K;
+  int r;
+};
+
+// Plane widths of a width r: b0 (low bits) and b1 (high bits, 0 if none).
+inline void plane_widths(int r, int& b0, int& b1) {
+  switch (r) {
+    case 8: b0 = 8; b1 = 0; return;
+    case 6: b0 = 4; b1 = 2; return;
+    case 4: b0 = 4; b1 = 0; return;
+    case 3: b0 = 2; b1 = 1; return;
+    case 2: b0 = 2; b1 = 0; return;
+    default: b0 = 0; b1 = 0; return;
+  }
+}
+
+// Per-(device, stream) scratch owned by the library.
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+// Returns a workspace of at least `bytes` for the current device and
+// `stream`, growing it if needed (growth synchronizes the device).
+cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out);
+// Device error word of the current device (zero-initialized).
+cudaError_t get_error_word(uint32_t** out);
+uint64_t wait_limit_ns();
+int sm_count();
+
+cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
+                            float* alpha, float* zero, cudaStream_t stream, int sms);
+cudaError_t launch_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* packed,
+                              cudaStream_t stream, int sms);
+
+// Decode path (M <= 32): plans, stages activations and launches the
+// persistent stream-K GEMV over all jobs (at most kGemvMaxLinears).
+constexpr int kGemvMaxLinears = 256;
+cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream);
+
+// Prefill path (M > 32): tcgen05 GEMM for one linear.
+cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);
+
+}  // namespace mq

@@ -1,0 +1,109 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/mq.h declares, computes sizes, and rejects bad arguments on the host
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nested_bit_weight_int8_b200 as mq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "mq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for want in ["mq_quantize_int8", "mq_slice_pack", "mq_linear", "mq_stack_forward",
+                 "mq_packed_bytes", "mq_last_error"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(mq.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(mq.EXPORTED) == set(_declared_functions())
+
+
+def test_version():
+    assert mq.version() > 0
+
+
+@pytest.mark.parametrize("r", [8, 6, 4, 3, 2])
+def test_packed_bytes(r):
+    assert mq.packed_bytes(14336, 4096, r) == 14336 * 4096 * r // 8
+    assert mq.packed_bytes(1, 32, r) == 4 * r
+
+
+def test_packed_bytes_rejects():
+    assert mq.packed_bytes(4, 48, 4) == 0      # K % 32
+    assert mq.packed_bytes(4, 64, 5) == 0      # r
+    assert mq.packed_bytes(0, 64, 4) == 0
+    assert mq.packed_bytes(4, 0, 4) == 0
+
+
+FAKE = 1 << 20  # an aligned non-null address; never dereferenced by rejected calls
+
+
+@pytest.mark.parametrize("args,what", [
+    ((FAKE, 1, 64, 256, FAKE, FAKE, FAKE, 4, FAKE, None), "ok-shape-bad-r"),
+])
+def test_linear_rejects_bad_width(args, what):
+    x, M, K, p, a, z, N, r, y, s = args
+    for bad_r in [0, 1, 5, 7, 9, 16]:
+        st = mq.raw_status("mq_linear", x, M, K, p, a, z, N, bad_r, y, s)
+        assert st == mq.MQ_ERR_INVALID_ARG
+        assert "r=" in mq.last_error()
+
+
+def test_linear_rejects_bad_shapes_and_pointers():
+    F = FAKE
+    cases = [
+        (F, 0, 256, F, F, F, 64, 4, F),      # M = 0
+        (F, 1, 96, F, F, F, 64, 4, F),       # K % 128
+        (F, 1, 0, F, F, F, 64, 4, F),        # K = 0
+        (F, 1, 256, F, F, F, 0, 4, F),       # N = 0
+        (None, 1, 256, F, F, F, 64, 4, F),   # null x
+        (F, 1, 256, None, F, F, 64, 4, F),   # null packed
+        (F + 8, 1, 256, F, F, F, 64, 4, F),  # misaligned x
+        (F, 1, 256, F + 4, F, F, 64, 4, F),  # misaligned packed
+        (F, 1, 256, F, F + 2, F, 64, 4, F),  # misaligned alpha
+    ]
+    for c in cases:
+        assert mq.raw_status("mq_linear", *c, None) == mq.MQ_ERR_INVALID_ARG, c
+        assert mq.last_error()
+
+
+def test_slice_pack_rejects():
+    F = FAKE
+    assert mq.raw_status("mq_slice_pack", F, 4, 48, 4, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_slice_pack", F, 4, 64, 5, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_slice_pack", None, 4, 64, 4, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_slice_pack", F + 1, 4, 64, 4, F, None) == mq.MQ_ERR_INVALID_ARG
+
+
+def test_quantize_rejects():
+    F = FAKE
+    assert mq.raw_status("mq_quantize_int8", F, 7, 4, 64, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8", F, 1, 0, 64, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8", None, 1, 4, 64, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8", F + 2, 0, 4, 64, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+
+
+def test_stack_rejects_bad_layers():
+    F = FAKE
+    lins = [(F, F, F, F, F, 64, 256)]
+    with pytest.raises(mq.MQError) as e:
+        mq.stack_forward(lins, [3], [4, 4], 1)
+    assert e.value.status == mq.MQ_ERR_INVALID_ARG
+    with pytest.raises(mq.MQError):
+        mq.stack_forward(lins, [0], [5], 1)        # width 5
+    with pytest.raises(mq.MQError):
+        mq.stack_forward(lins, [0], [4], 33)       # M > 32
