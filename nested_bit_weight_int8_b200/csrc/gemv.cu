@@ -9,10 +9,10 @@
 // so every CTA streams the same number of units whatever the shapes. Partial
 // row sums are added into y with fp32 atomics; the prep kernel zeroes y.
 //
-// CTA = 4 consumer warps + 1 producer warp. The producer stages each unit in
+// CTA = 8 consumer warps + 1 producer warp. The producer stages each unit in
 // shared memory with 1-D bulk copies (cp.async.bulk, one per row and plane)
 // plus one copy of the activation block, signalling an mbarrier. Each
-// consumer warp owns 2 tiles of 16 rows and runs mma.sync m16n8k16 (bf16 in,
+// consumer warp owns one tile of 16 rows and runs mma.sync m16n8k16 (bf16 in,
 // fp32 accumulate) with the weights as the A operand and the batch (M <= 32,
 // n8 tiles) as B.
 //
@@ -33,6 +33,7 @@
 #include <cstdint>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <utility>
 #include <vector>
 
@@ -42,12 +43,15 @@
 namespace mq {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kTilesPerWarp = 2;
+constexpr int kConsumerWarps = 8;
+constexpr int kTilesPerWarp = 1;
+constexpr int kRowsPerWarp = 16 * kTilesPerWarp;
 constexpr int kRowsPerUnit = kConsumerWarps * kTilesPerWarp * 16;  // 128
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxStages = 8;
-constexpr int kBarrierBytes = 256;
+constexpr int kBarrierBytes = 256;  // barriers, abort flag; last 64 bytes: zero block
+constexpr int kMaxDynSmem = 227 * 1024;
+constexpr size_t kStageBudget = 110 * 1024;
 
 // Per-linear descriptor, passed by value in the kernel parameters.
 struct LinDesc {
@@ -63,6 +67,10 @@ struct LinDesc {
 
 template <int CAP>
 struct GemvParams {
+  // Tensor maps of the planes (plane 0, plane 1 per linear): inline for small
+  // launches, else in a device table built once per distinct stack.
+  CUtensorMap maps[CAP <= 8 ? 2 * CAP : 1];
+  const CUtensorMap* map_table;
   int n_lin, M, total_units, stages;
   uint32_t stage_bytes, off_plane1, off_x;
   int pitch0, pitch1;
@@ -71,15 +79,14 @@ struct GemvParams {
   LinDesc lin[CAP];
 };
 
-// Geometry of one width: the high-plane width b1 (0 if one plane), the
-// 8-code activation groups per 16-byte low-plane chunk (W8) and the MMAs fed
-// by one group (MPG: 2 when each code fills one k-slot, 4 when it fills two).
+// Geometry of one width: plane widths, 8-code activation groups per 16-byte
+// low-plane chunk (W8).
 template <int R> struct Geo;
-template <> struct Geo<2> { static constexpr int b1 = 0, W8 = 8, MPG = 2; };
-template <> struct Geo<4> { static constexpr int b1 = 0, W8 = 4, MPG = 2; };
-template <> struct Geo<8> { static constexpr int b1 = 0, W8 = 2, MPG = 4; };
-template <> struct Geo<3> { static constexpr int b1 = 1, W8 = 8, MPG = 4; };
-template <> struct Geo<6> { static constexpr int b1 = 2, W8 = 4, MPG = 4; };
+template <> struct Geo<2> { static constexpr int b0 = 2, b1 = 0, W8 = 8; };
+template <> struct Geo<4> { static constexpr int b0 = 4, b1 = 0, W8 = 4; };
+template <> struct Geo<8> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
+template <> struct Geo<3> { static constexpr int b0 = 2, b1 = 1, W8 = 8; };
+template <> struct Geo<6> { static constexpr int b0 = 4, b1 = 2, W8 = 4; };
 
 __device__ __forceinline__ void plane_widths_dev(int r, int& b0, int& b1) {
   b0 = (r == 8) ? 8 : (r == 4 || r == 6) ? 4 : 2;
@@ -89,56 +96,69 @@ __device__ __forceinline__ void plane_widths_dev(int r, int& b0, int& b1) {
 template <int SIG>
 __device__ __forceinline__ uint32_t shift_to(uint32_t w) {
   if constexpr (SIG < 0) return w << (-SIG);
+  else if constexpr (SIG == 0) return w;
   else return w >> SIG;
 }
 
-// bf16x2 magic constants 2^e in both halves.
+// (a & mask) | magic in one LOP3: both constants travel in registers, so the
+// instruction needs no second immediate.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+  return d;
+}
+
+// bf16x2 powers of two 2^e in both halves (OR-ing a code into the mantissa
+// gives 2^e + code * 2^(e-7+p) exactly).
 constexpr uint32_t kMag4 = 0x40804080u, kMag8 = 0x41004100u, kMag16 = 0x41804180u,
                    kMag32 = 0x42004200u, kMag64 = 0x42804280u, kMag128 = 0x43004300u,
                    kMag256 = 0x43804380u;
+constexpr uint32_t kMaskP3b2 = 0x00180018u, kMaskP5b2 = 0x00600060u, kMaskP3b4 = 0x00780078u,
+                   kMaskP0b4 = 0x000F000Fu;
 
-// Decodes the two A registers (x0: slots {2t, 2t+1}; x1: slots {2t+8, 2t+9})
-// of MMA J for one weight row from its low-plane words lo[4] and high-plane
-// words hi[2]. Each register holds the bf16 values of two neighbouring codes.
-template <int R, int J>
-__device__ __forceinline__ void decode_pair(const uint32_t (&lo)[4], const uint32_t (&hi)[2],
+// Decoded A registers of one MMA for one weight row: x0 fills k-slots
+// {2t, 2t+1}, x1 fills {2t+8, 2t+9}. PLANE 0 is the low plane, 1 the high
+// plane; Q is the 8-code group of the chunk, HF the 4-code half of it.
+template <int R, int PLANE, int Q, int HF>
+__device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint32_t (&hi)[2],
                                             uint32_t& x0, uint32_t& x1) {
-  if constexpr (R == 2) {
-    // codes 4J..4J+3: pair 2jj at half-bit 4jj -> bits 3-4 (16+c), pair 2jj+1 -> bits 5-6 (4+c)
-    constexpr int jj = J % 4;
-    const uint32_t sh = shift_to<4 * jj - 3>(lo[J / 4]);
-    x0 = (sh & 0x00180018u) | kMag16;
-    x1 = (sh & 0x00600060u) | kMag4;
-  } else if constexpr (R == 4) {
-    // codes 4J..4J+3: pairs pa, pa+1 at half-bits 4pa, 4pa+4 -> bits 3-6 (16+c)
-    constexpr int pa = 2 * (J % 2);
-    const uint32_t w = lo[J / 2];
-    x0 = (shift_to<4 * pa - 3>(w) & 0x00780078u) | kMag16;
-    x1 = (shift_to<4 * (pa + 1) - 3>(w) & 0x00780078u) | kMag16;
+  if constexpr (R == 2 || (R == 3 && PLANE == 0)) {
+    // 2-bit codes, word = 16 codes; pairs 2j, 2j+1 (j = 2(Q%2)+HF) at half-bits
+    // 4j, 4j+2 -> bits 3-4 (16 + c) and bits 5-6 (4 + c) after one shift.
+    constexpr int j = 2 * (Q % 2) + HF;
+    const uint32_t sh = shift_to<4 * j - 3>(lo[Q / 2]);
+    x0 = and_or(sh, kMaskP3b2, kMag16);
+    x1 = and_or(sh, kMaskP5b2, kMag4);
+  } else if constexpr (R == 4 || (R == 6 && PLANE == 0)) {
+    // 4-bit codes, word = 8 codes; pairs 2HF, 2HF+1 at half-bits 8HF, 8HF+4 -> bits 3-6 (16 + c)
+    const uint32_t w = lo[Q];
+    x0 = and_or(shift_to<8 * HF - 3>(w), kMaskP3b4, kMag16);
+    x1 = and_or(shift_to<8 * HF + 1>(w), kMaskP3b4, kMag16);
   } else if constexpr (R == 8) {
-    // codes 2J, 2J+1 (bytes): low nibble -> 128+l, high nibble -> 256+16h
-    const uint32_t d = __byte_perm(lo[J / 2], 0u, (J % 2) ? 0x4342u : 0x4140u);
-    x0 = (d & 0x000F000Fu) | kMag128;
-    x1 = ((d >> 1) & 0x00780078u) | kMag256;
+    // bytes c0..c3 of one word; registers pair (c0, c2) and (c1, c3):
+    // low nibble -> 128 + l (bits 0-3), high nibble -> 256 + 16h (bits 3-6)
+    const uint32_t w = lo[2 * Q + HF];
+    if constexpr (PLANE == 0) {
+      x0 = and_or(w, kMaskP0b4, kMag128);
+      x1 = and_or(w >> 8, kMaskP0b4, kMag128);
+    } else {
+      x0 = and_or(w >> 1, kMaskP3b4, kMag256);
+      x1 = and_or(w >> 9, kMaskP3b4, kMag256);
+    }
   } else if constexpr (R == 3) {
-    // codes 2J, 2J+1: low 2-bit plane -> 16+c or 4+c; high 1-bit plane (weight 4)
-    constexpr int pl = J % 8;
-    const uint32_t sl = shift_to<4 * (pl / 2) - 3>(lo[J / 8]);
-    if constexpr (pl % 2 == 0) x0 = (sl & 0x00180018u) | kMag16;
-    else x0 = (sl & 0x00600060u) | kMag4;
-    constexpr int ph = J % 16;
-    constexpr int p = 3 + ph % 4;
-    constexpr uint32_t mask = (1u << p) | (1u << (16 + p));
-    constexpr uint32_t mag = (ph % 4 == 0) ? kMag64 : (ph % 4 == 1) ? kMag32 : (ph % 4 == 2) ? kMag16 : kMag8;
-    x1 = (shift_to<4 * (ph / 4) - 3>(hi[J / 16]) & mask) | mag;
-  } else {  // R == 6
-    // codes 2J, 2J+1: low 4-bit plane -> 16+c; high 2-bit plane (weight 16) -> 256+16h or 64+16h
-    constexpr int pl = J % 4;
-    x0 = (shift_to<4 * pl - 3>(lo[J / 4]) & 0x00780078u) | kMag16;
-    constexpr int ph = J % 8;
-    const uint32_t sh = shift_to<4 * (ph / 2) - 3>(hi[J / 8]);
-    if constexpr (ph % 2 == 0) x1 = (sh & 0x00180018u) | kMag256;
-    else x1 = (sh & 0x00600060u) | kMag64;
+    // high 1-bit plane (weight 4), word = 32 codes; pairs P = 4(Q%4)+2HF, +1 at
+    // half-bit P; one shift puts the group's 4 pairs at bits 3..6 (64/32/16/8 + 4h)
+    const uint32_t sh = shift_to<4 * (Q % 4) - 3>(hi[Q / 4]);
+    constexpr int p0 = 3 + 2 * HF;
+    constexpr uint32_t m0 = (1u << p0) | (1u << (16 + p0));
+    constexpr uint32_t m1 = (1u << (p0 + 1)) | (1u << (17 + p0));
+    x0 = and_or(sh, m0, HF == 0 ? kMag64 : kMag16);
+    x1 = and_or(sh, m1, HF == 0 ? kMag32 : kMag8);
+  } else {  // R == 6, high 2-bit plane (weight 16), word = 16 codes
+    constexpr int j = 2 * (Q % 2) + HF;
+    const uint32_t sh = shift_to<4 * j - 3>(hi[Q / 2]);
+    x0 = and_or(sh, kMaskP3b2, kMag256);
+    x1 = and_or(sh, kMaskP5b2, kMag64);
   }
 }
 
@@ -153,143 +173,167 @@ __device__ __forceinline__ void offset_coeffs(int r, float (&c)[4]) {
   }
 }
 
-template <int R, int MMA_J, int NT>
-__device__ __forceinline__ void mma_step(const uint32_t (&lo)[kTilesPerWarp][2][4],
-                                         const uint32_t (&hi)[kTilesPerWarp][2][2],
-                                         const uint4 (&xb)[NT],
-                                         float (&ch)[kTilesPerWarp][NT][2][4]) {
-  using G = Geo<R>;
-  uint32_t b0[NT], b1[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const uint32_t comp[4] = {xb[nt].x, xb[nt].y, xb[nt].z, xb[nt].w};
-    if constexpr (G::MPG == 2) {
-      b0[nt] = comp[2 * (MMA_J % 2)];
-      b1[nt] = comp[2 * (MMA_J % 2) + 1];
-    } else {
-      b0[nt] = comp[MMA_J % 4];
-      b1[nt] = b0[nt];
-    }
-  }
-#pragma unroll
-  for (int tau = 0; tau < kTilesPerWarp; ++tau) {
-    uint32_t a0, a1, a2, a3;
-    decode_pair<R, MMA_J>(lo[tau][0], hi[tau][0], a0, a2);
-    decode_pair<R, MMA_J>(lo[tau][1], hi[tau][1], a1, a3);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(ch[tau][nt][MMA_J & 1], a0, a1, a2, a3, b0[nt], b1[nt]);
-  }
-}
-
+// All MMAs of one 8-code activation group: for each 4-code half and each
+// plane, one m16n8k16 per batch tile, the B registers shared by the planes.
 template <int R, int NT, int Q>
-__device__ __forceinline__ void group_steps(const uint32_t (&lo)[kTilesPerWarp][2][4],
-                                            const uint32_t (&hi)[kTilesPerWarp][2][2],
-                                            const uint8_t* xq, uint32_t xstride, bool (&mval)[NT],
-                                            float (&ch)[kTilesPerWarp][NT][2][4]) {
-  using G = Geo<R>;
+__device__ __forceinline__ void group_mmas(const uint32_t (&lo)[2][4], const uint32_t (&hi)[2][2],
+                                           const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
+                                           int gbase, float (&ch)[NT][2][4]) {
   uint4 xb[NT];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-    xb[nt] = mval[nt] ? *reinterpret_cast<const uint4*>(xq + nt * xstride) : make_uint4(0, 0, 0, 0);
-  if constexpr (G::MPG >= 1) mma_step<R, Q * G::MPG + 0, NT>(lo, hi, xb, ch);
-  if constexpr (G::MPG >= 2) mma_step<R, Q * G::MPG + 1, NT>(lo, hi, xb, ch);
-  if constexpr (G::MPG >= 3) mma_step<R, Q * G::MPG + 2, NT>(lo, hi, xb, ch);
-  if constexpr (G::MPG >= 4) mma_step<R, Q * G::MPG + 3, NT>(lo, hi, xb, ch);
+  for (int nt = 0; nt < NT; ++nt) {
+    const uint32_t a = xaddr[nt] + static_cast<uint32_t>(gbase + Q) * xstep[nt];
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(xb[nt].x), "=r"(xb[nt].y), "=r"(xb[nt].z), "=r"(xb[nt].w)
+                 : "r"(a));
+  }
+  // two operand planes for r = 3, 6 (low/high bit planes) and r = 8 (low/high nibbles)
+  constexpr int NPL = (Geo<R>::b1 != 0 || R == 8) ? 2 : 1;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+    for (int pl = 0; pl < NPL; ++pl) {
+      uint32_t a0, a1, a2, a3;
+      if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[0], hi[0], a0, a2); decode_quad<R, 0, Q, 0>(lo[1], hi[1], a1, a3); }
+      if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[0], hi[0], a0, a2); decode_quad<R, 1, Q, 0>(lo[1], hi[1], a1, a3); }
+      if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[0], hi[0], a0, a2); decode_quad<R, 0, Q, 1>(lo[1], hi[1], a1, a3); }
+      if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[0], hi[0], a0, a2); decode_quad<R, 1, Q, 1>(lo[1], hi[1], a1, a3); }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t b0 = hf ? xb[nt].z : xb[nt].x;
+        const uint32_t b1 = hf ? xb[nt].w : xb[nt].y;
+        mma_bf16_16816(ch[nt][(2 * Q + hf + pl) & 1], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
 }
 
 template <int R, int NT, int... Qs>
-__device__ __forceinline__ void all_groups(const uint32_t (&lo)[kTilesPerWarp][2][4],
-                                           const uint32_t (&hi)[kTilesPerWarp][2][2],
-                                           const uint8_t* xs, int M, uint32_t xstride_q,
-                                           uint32_t xstride_nt, bool (&mval)[NT],
-                                           float (&ch)[kTilesPerWarp][NT][2][4],
+__device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[2][4], const uint32_t (&hi)[2][2],
+                                           const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
+                                           int gbase, float (&ch)[NT][2][4],
                                            std::integer_sequence<int, Qs...>) {
-  (group_steps<R, NT, Qs>(lo, hi, xs + Qs * xstride_q, xstride_nt, mval, ch), ...);
+  (group_mmas<R, NT, Qs>(lo, hi, xaddr, xstep, gbase, ch), ...);
 }
 
-// Processes one staged unit for this warp's two 16-row tiles.
-template <int R, int NT>
+// One staged unit for this warp's 16-row tile. All NSUB sub-steps are
+// unrolled and their plane loads issued first. Sub-steps past the unit's
+// valid codes read zero-filled planes and zero activations and add nothing.
+// Activation group q of chunk 4s+t for batch row m sits at
+// ((((s*W8 + q)*M + m)*4 + t) * 16) bytes of the staged block; lanes whose
+// batch row is past M read a zero block instead (step 0).
+template <int R, int NT, int NSUB>
 __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* st1,
-                                             const uint8_t* stx, int pitch0, int pitch1,
-                                             int nsub, int M, int warp, int lane,
-                                             float (&ch)[kTilesPerWarp][NT][2][4]) {
+                                             const uint32_t (&xaddr)[NT],
+                                             const uint32_t (&xstep)[NT], int pitch0, int pitch1,
+                                             int warp, int lane, float (&ch)[NT][2][4]) {
   using G = Geo<R>;
   const int g = lane >> 2, t = lane & 3;
-  bool mval[NT];
+  uint32_t lo[NSUB][2][4];
+  uint32_t hi[NSUB][2][2];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) mval[nt] = (nt * 8 + g) < M;
-  for (int s = 0; s < nsub; ++s) {
+  for (int s = 0; s < NSUB; ++s) {
     const int ci = 4 * s + t;  // this thread's 16-byte chunk of the low plane
-    uint32_t lo[kTilesPerWarp][2][4];
-    uint32_t hi[kTilesPerWarp][2][2];
 #pragma unroll
-    for (int tau = 0; tau < kTilesPerWarp; ++tau) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = warp * 32 + tau * 16 + g + 8 * h;
-        const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * pitch0 + ci * 16);
-        lo[tau][h][0] = v.x; lo[tau][h][1] = v.y; lo[tau][h][2] = v.z; lo[tau][h][3] = v.w;
-        if constexpr (G::b1 != 0) {
-          const uint2 u = *reinterpret_cast<const uint2*>(st1 + row * pitch1 + ci * 8);
-          hi[tau][h][0] = u.x; hi[tau][h][1] = u.y;
-        } else {
-          hi[tau][h][0] = 0; hi[tau][h][1] = 0;
-        }
+    for (int h = 0; h < 2; ++h) {
+      const int row = warp * kRowsPerWarp + g + 8 * h;
+      const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * pitch0 + ci * 16);
+      lo[s][h][0] = v.x; lo[s][h][1] = v.y; lo[s][h][2] = v.z; lo[s][h][3] = v.w;
+      if constexpr (G::b1 != 0) {
+        const uint2 u = *reinterpret_cast<const uint2*>(st1 + row * pitch1 + ci * 8);
+        hi[s][h][0] = u.x; hi[s][h][1] = u.y;
+      } else {
+        hi[s][h][0] = 0; hi[s][h][1] = 0;
       }
     }
-    // Activation group q of chunk ci for batch row m sits at
-    // ((((s*W8 + q)*M + m)*4 + t) * 16) bytes of the staged block.
-    const uint8_t* xs = stx + ((static_cast<uint32_t>(s * G::W8) * M + g) * 4 + t) * 16;
-    all_groups<R, NT>(lo, hi, xs, M, static_cast<uint32_t>(M) * 64u, 8u * 64u, mval, ch,
+  }
+#pragma unroll
+  for (int s = 0; s < NSUB; ++s)
+    chunk_mmas<R, NT>(lo[s], hi[s], xaddr, xstep, s * G::W8, ch,
                       std::make_integer_sequence<int, G::W8>{});
+}
+
+// The current linear of a CTA's walk over its unit range, cached in registers.
+struct Cursor {
+  int l, rb, kc;          // linear, row block, k-chunk of the current unit
+  int nrb, n_kc, r, N;    // of linear l
+};
+
+template <int CAP>
+__device__ __forceinline__ void cursor_load(const GemvParams<CAP>& p, Cursor& c) {
+  const LinDesc& L = p.lin[c.l];
+  c.n_kc = L.n_kc;
+  c.nrb = (L.N + kRowsPerUnit - 1) / kRowsPerUnit;
+  c.r = L.r;
+  c.N = L.N;
+}
+
+template <int CAP>
+__device__ __forceinline__ void cursor_init(const GemvParams<CAP>& p, int u, Cursor& c) {
+  int l = 0;
+  while (l + 1 < p.n_lin && u >= p.lin[l + 1].unit_begin) ++l;
+  c.l = l;
+  cursor_load(p, c);
+  const int local = u - p.lin[l].unit_begin;
+  c.rb = local / c.n_kc;
+  c.kc = local - c.rb * c.n_kc;
+}
+
+template <int CAP>
+__device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c) {
+  if (++c.kc == c.n_kc) {
+    c.kc = 0;
+    if (++c.rb == c.nrb) {
+      c.rb = 0;
+      ++c.l;
+      if (c.l < p.n_lin) cursor_load(p, c);
+    }
   }
 }
 
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, int warp, int lane,
-                           float (&tot)[kTilesPerWarp][NT][4]) {
+                           float (&tot)[NT][4]) {
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
   float c[4];
   offset_coeffs(L.r, c);
 #pragma unroll
-  for (int tau = 0; tau < kTilesPerWarp; ++tau) {
+  for (int h = 0; h < 2; ++h) {
+    const int n = rb * kRowsPerUnit + warp * kRowsPerWarp + g + 8 * h;
+    if (n >= L.N) continue;
+    const float a = L.alpha[n], z = L.zero[n];
+    const float A = a * scale, B = a * z;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int n = rb * kRowsPerUnit + warp * 32 + tau * 16 + g + 8 * h;
-      if (n >= L.N) continue;
-      const float a = L.alpha[n], z = L.zero[n];
-      const float A = a * scale, B = a * z;
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int m = nt * 8 + 2 * t + e;
-          if (m >= p.M) continue;
-          float v = tot[tau][nt][2 * h + e];
-          if (kc0 == 0) {
-            const float* P = L.psum + m * 4;
-            const float O = c[0] * P[0] + c[1] * P[1] + c[2] * P[2] + c[3] * P[3];
-            const float Sx = (P[0] + P[1]) + (P[2] + P[3]);
-            v = A * (v - O) - B * Sx;
-          } else {
-            v = A * v;
-          }
-          atomicAdd(L.y + static_cast<int64_t>(m) * L.N + n, v);
+      for (int e = 0; e < 2; ++e) {
+        const int m = nt * 8 + 2 * t + e;
+        if (m >= p.M) continue;
+        float v = tot[nt][2 * h + e];
+        if (kc0 == 0) {
+          const float* P = L.psum + m * 4;
+          const float O = c[0] * P[0] + c[1] * P[1] + c[2] * P[2] + c[3] * P[3];
+          const float Sx = (P[0] + P[1]) + (P[2] + P[3]);
+          v = A * (v - O) - B * Sx;
+        } else {
+          v = A * v;
         }
+        atomicAdd(L.y + static_cast<int64_t>(m) * L.N + n, v);
       }
     }
   }
 }
 
 template <int NT, int CAP>
-__global__ void __launch_bounds__(kGemvThreads, 2)
+__global__ void __launch_bounds__(kGemvThreads, (NT <= 2 ? 2 : 1))
 gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
+  uint8_t* zero_block = smem + kBarrierBytes - 64;  // 64 zero bytes read by lanes past M
   uint8_t* stages = smem + kBarrierBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
@@ -302,84 +346,101 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
     *s_abort = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(zero_block)[threadIdx.x] = 0u;
   __syncthreads();
 
-  const int64_t G = gridDim.x, c = blockIdx.x;
-  const int u0 = static_cast<int>(int64_t(p.total_units) * c / G);
-  const int u1 = static_cast<int>(int64_t(p.total_units) * (c + 1) / G);
-
-  // Activations, class sums and the zeroed outputs come from the prep kernel.
-  pdl_wait_primary();
+  const int64_t G = gridDim.x, cta = blockIdx.x;
+  const int u0 = static_cast<int>(int64_t(p.total_units) * cta / G);
+  const int u1 = static_cast<int>(int64_t(p.total_units) * (cta + 1) / G);
+  if (u0 >= u1) return;
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    int l = 0, issued = 0;
+    // Weight boxes do not depend on the prep kernel, so the first stages'
+    // boxes are requested before waiting for it; their activation blocks
+    // follow once the prep grid has finished.
     bool aborted = false;
-    for (int u = u0; u < u1; ++u, ++issued) {
-      const int s = issued % S;
-      if (issued >= S) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_bounded(&empty[s], ((issued / S) - 1) & 1, p.wait_ns);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) {
-          if (lane == 0) { atomicOr(p.err, kErrWaitEmpty); *s_abort = 1; }
+    int issued = 0;
+    if (lane == 0) {
+      Cursor c;
+      cursor_init(p, u0, c);
+      Cursor pre_c = c;
+      auto issue_weights = [&](const Cursor& cc, int s) {
+        int b0, b1;
+        plane_widths_dev(cc.r, b0, b1);
+        uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+        const CUtensorMap* tm = p.map_table ? p.map_table + 2 * cc.l : &p.maps[2 * cc.l];
+        const uint32_t box = kRowsPerUnit * (p.pitch0 + (b1 ? p.pitch1 : 0));
+        const uint32_t bytesx = static_cast<uint32_t>(p.M * p.lin[cc.l].kc * 2);
+        // One 2-D box per plane (128 rows x the unit's bytes; rows past N and
+        // bytes past K read as zero) plus the unit's activation block.
+        mbar_arrive_expect_tx(&full[s], box + bytesx);
+        tma_load_2d(st, tm, cc.kc * p.pitch0, cc.rb * kRowsPerUnit, &full[s]);
+        if (b1) tma_load_2d(st + p.off_plane1, tm + 1, cc.kc * p.pitch1, cc.rb * kRowsPerUnit, &full[s]);
+      };
+      auto issue_x = [&](const Cursor& cc, int s) {
+        const LinDesc& L = p.lin[cc.l];
+        const uint32_t bytesx = static_cast<uint32_t>(p.M * L.kc * 2);
+        uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+        bulk_g2s(st + p.off_x, L.xf + int64_t(cc.kc) * bytesx, bytesx, &full[s]);
+      };
+      const int pre = min(S, u1 - u0);
+      for (int i = 0; i < pre; ++i) { issue_weights(c, i); cursor_next(p, c); }
+      pdl_wait_primary();
+      for (int i = 0; i < pre; ++i) { issue_x(pre_c, i); cursor_next(p, pre_c); }
+      issued = pre;
+      for (int u = u0 + pre; u < u1; ++u, ++issued) {
+        const int s = issued % S;
+        if (!mbar_wait_bounded(&empty[s], ((issued / S) - 1) & 1, p.wait_ns)) {
+          atomicOr(p.err, kErrWaitEmpty);
+          *s_abort = 1;
           aborted = true;
           break;
         }
+        if (*s_abort) { aborted = true; break; }
+        issue_weights(c, s);
+        issue_x(c, s);
+        cursor_next(p, c);
       }
-      if (*s_abort) { aborted = true; break; }
-      while (l + 1 < p.n_lin && u >= p.lin[l + 1].unit_begin) ++l;
-      const LinDesc& L = p.lin[l];
-      const int local = u - L.unit_begin;
-      const int rb = local / L.n_kc, kc = local - rb * L.n_kc;
-      const int ncodes = min(L.kc, L.K - kc * L.kc);
-      const int rows = min(kRowsPerUnit, L.N - rb * kRowsPerUnit);
-      int b0, b1;
-      plane_widths_dev(L.r, b0, b1);
-      const uint32_t bytes0 = static_cast<uint32_t>(ncodes * b0 / 8);
-      const uint32_t bytes1 = static_cast<uint32_t>(ncodes * b1 / 8);
-      const uint32_t bytesx = static_cast<uint32_t>(p.M * L.kc * 2);
-      uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
-      if (lane == 0)
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(rows) * (bytes0 + bytes1) + bytesx);
-      __syncwarp();
-      const int64_t row0 = int64_t(rb) * kRowsPerUnit;
-      const int64_t gp0 = int64_t(L.K) * b0 / 8, gp1 = int64_t(L.K) * b1 / 8;
-      const int ncopies = rows * (b1 ? 2 : 1) + 1;
-      for (int cidx = lane; cidx < ncopies; cidx += 32) {
-        if (cidx == ncopies - 1) {
-          bulk_g2s(st + p.off_x, L.xf + int64_t(kc) * bytesx, bytesx, &full[s]);
-        } else if (cidx < rows) {
-          bulk_g2s(st + cidx * p.pitch0,
-                   L.plane0 + (row0 + cidx) * gp0 + int64_t(kc) * (L.kc * b0 / 8), bytes0, &full[s]);
-        } else {
-          const int i = cidx - rows;
-          bulk_g2s(st + p.off_plane1 + i * p.pitch1,
-                   L.plane1 + (row0 + i) * gp1 + int64_t(kc) * (L.kc * b1 / 8), bytes1, &full[s]);
+      if (aborted) {
+        // Leave no bulk copy in flight: wait for the last issue of every stage.
+        const int first = issued > S ? issued - S : 0;
+        for (int j = first; j < issued; ++j) {
+          if (!mbar_wait_bounded(&full[j % S], (j / S) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
         }
       }
-    }
-    if (aborted && lane == 0) {
-      // Leave no bulk copy in flight: wait for the last issue of every stage.
-      const int first = issued > S ? issued - S : 0;
-      for (int j = first; j < issued; ++j) {
-        if (!mbar_wait_bounded(&full[j % S], (j / S) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
-      }
+    } else {
+      pdl_wait_primary();
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  float ch[kTilesPerWarp][NT][2][4];
-  float tot[kTilesPerWarp][NT][4];
+  // Class sums and the zeroed outputs come from the prep kernel.
+  pdl_wait_primary();
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t xaddr[NT], xstep[NT];
+  const uint32_t zero_addr = smem_u32(zero_block) + t * 16;
 #pragma unroll
-  for (int a = 0; a < kTilesPerWarp; ++a)
+  for (int nt = 0; nt < NT; ++nt) {
+    const int m = nt * 8 + g;
+    xaddr[nt] = zero_addr;
+    xstep[nt] = 0;
+    if (m < p.M) {
+      xaddr[nt] = static_cast<uint32_t>((m * 4 + t) * 16);  // + stage x base, per unit
+      xstep[nt] = static_cast<uint32_t>(p.M) * 64u;
+    }
+  }
+  float ch[NT][2][4];
+  float tot[NT][4];
 #pragma unroll
-    for (int b = 0; b < NT; ++b)
+  for (int b = 0; b < NT; ++b)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) { ch[a][b][0][i] = 0.f; ch[a][b][1][i] = 0.f; tot[a][b][i] = 0.f; }
+    for (int i = 0; i < 4; ++i) { ch[b][0][i] = 0.f; ch[b][1][i] = 0.f; tot[b][i] = 0.f; }
 
-  int l = 0, cur_l = -1, cur_rb = -1, cur_kc0 = 0;
+  Cursor c;
+  cursor_init(p, u0, c);
+  int cur_l = c.l, cur_rb = c.rb, cur_kc0 = c.kc;
   bool aborted = false;
   int it = 0;
   for (int u = u0; u < u1; ++u, ++it) {
@@ -389,51 +450,46 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       aborted = true;
       break;
     }
-    while (l + 1 < p.n_lin && u >= p.lin[l + 1].unit_begin) ++l;
-    const LinDesc& L = p.lin[l];
-    const int local = u - L.unit_begin;
-    const int rb = local / L.n_kc, kc = local - rb * L.n_kc;
-    if (l != cur_l || rb != cur_rb) {
-      if (cur_l >= 0) flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
+    if (c.l != cur_l || c.rb != cur_rb) {
+      flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
 #pragma unroll
-      for (int a = 0; a < kTilesPerWarp; ++a)
+      for (int b = 0; b < NT; ++b)
 #pragma unroll
-        for (int b = 0; b < NT; ++b)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) tot[a][b][i] = 0.f;
-      cur_l = l; cur_rb = rb; cur_kc0 = kc;
+        for (int i = 0; i < 4; ++i) tot[b][i] = 0.f;
+      cur_l = c.l; cur_rb = c.rb; cur_kc0 = c.kc;
     }
-    const int rows = min(kRowsPerUnit, L.N - rb * kRowsPerUnit);
-    if (warp * 32 < rows) {
-      const int ncodes = min(L.kc, L.K - kc * L.kc);
+    const int rows = c.N - c.rb * kRowsPerUnit;
+    if (warp * kRowsPerWarp < rows) {
       const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
-      int b0, b1;
-      plane_widths_dev(L.r, b0, b1);
-      const int per_sub = 512 / b0;  // codes covered by one sub-step (4 chunks of 16 bytes)
-      const int nsub = (ncodes + per_sub - 1) / per_sub;
-      switch (L.r) {
-        case 2: process_unit<2, NT>(st, st + p.off_plane1, st + p.off_x, p.pitch0, p.pitch1, nsub, p.M, warp, lane, ch); break;
-        case 4: process_unit<4, NT>(st, st + p.off_plane1, st + p.off_x, p.pitch0, p.pitch1, nsub, p.M, warp, lane, ch); break;
-        case 8: process_unit<8, NT>(st, st + p.off_plane1, st + p.off_x, p.pitch0, p.pitch1, nsub, p.M, warp, lane, ch); break;
-        case 3: process_unit<3, NT>(st, st + p.off_plane1, st + p.off_x, p.pitch0, p.pitch1, nsub, p.M, warp, lane, ch); break;
-        default: process_unit<6, NT>(st, st + p.off_plane1, st + p.off_x, p.pitch0, p.pitch1, nsub, p.M, warp, lane, ch); break;
+      const uint32_t xs = smem_u32(st + p.off_x);
+      uint32_t xa[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) xa[nt] = xstep[nt] ? xs + xaddr[nt] : xaddr[nt];
+      // Sub-steps per unit: the low plane holds 192 bytes per row per unit
+      // for M <= 8 (3 sub-steps of 64 bytes) and 64 bytes for larger M.
+      constexpr int NSUB = (NT == 1) ? 3 : 1;
+      switch (c.r) {
+        case 2: process_unit<2, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
+        case 4: process_unit<4, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
+        case 8: process_unit<8, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
+        case 3: process_unit<3, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
+        default: process_unit<6, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
       }
       // Fold the two MMA chains into the row totals once per unit.
 #pragma unroll
-      for (int a = 0; a < kTilesPerWarp; ++a)
+      for (int b = 0; b < NT; ++b)
 #pragma unroll
-        for (int b = 0; b < NT; ++b)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            tot[a][b][i] += ch[a][b][0][i] + ch[a][b][1][i];
-            ch[a][b][0][i] = 0.f;
-            ch[a][b][1][i] = 0.f;
-          }
+        for (int i = 0; i < 4; ++i) {
+          tot[b][i] += ch[b][0][i] + ch[b][1][i];
+          ch[b][0][i] = 0.f;
+          ch[b][1][i] = 0.f;
+        }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    cursor_next(p, c);
   }
-  if (!aborted && cur_l >= 0) flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
+  if (!aborted) flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
 }
 
 // ------------------------------------------------------------------ prep
@@ -441,6 +497,7 @@ struct PrepLayout {
   const __nv_bfloat16* x;
   uint8_t* xf;
   int K, kc, w8, n_kc;
+  int perm02;  // byte planes pair codes (c0, c2), (c1, c3): store x0, x2, x1, x3
 };
 struct PrepSum {
   const __nv_bfloat16* x;
@@ -509,6 +566,11 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       const int k0 = kc * L.kc + grp * 8;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (k0 < L.K) v = *reinterpret_cast<const uint4*>(L.x + int64_t(m) * L.K + k0);
+      if (L.perm02) {
+        const uint32_t a = __byte_perm(v.x, v.y, 0x5410), b = __byte_perm(v.x, v.y, 0x7632);
+        const uint32_t c = __byte_perm(v.z, v.w, 0x5410), d = __byte_perm(v.z, v.w, 0x7632);
+        v = make_uint4(a, b, c, d);
+      }
       const int s = grp / (4 * L.w8);
       const int rem = grp % (4 * L.w8);
       const int t = rem / L.w8, q = rem % L.w8;
@@ -525,13 +587,43 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
   }
 }
 
-template <int NT>
-cudaError_t launch_gemv_nt(const GemvParams<kGemvMaxLinears>& gp, int grid, size_t smem,
-                           cudaStream_t stream) {
-  auto kern = gemv_streamk_kernel<NT, kGemvMaxLinears>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+// Per-(device, kernel instantiation) launch facts, computed once: the
+// dynamic shared-memory limit is raised to the largest stage plan and the
+// occupancy of each shared-memory size is remembered.
+struct KernelCache {
+  bool attr_set = false;
+  std::map<size_t, int> occ;
+};
+std::mutex g_cache_mutex;
+
+template <int NT, int CAP>
+cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int sms, int units,
+                        cudaStream_t stream) {
+  auto kern = gemv_streamk_kernel<NT, CAP>;
+  static std::map<int, KernelCache> caches;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int occ = 1;
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mutex);
+    KernelCache& kc = caches[dev];
+    if (!kc.attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kMaxDynSmem);
+      if (e != cudaSuccess) return e;
+      kc.attr_set = true;
+    }
+    auto it = kc.occ.find(smem);
+    if (it == kc.occ.end()) {
+      int blocks = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kGemvThreads, smem) != cudaSuccess ||
+          blocks < 1)
+        blocks = 1;
+      it = kc.occ.emplace(smem, blocks).first;
+    }
+    occ = it->second;
+  }
+  const int grid = std::max(1, std::min(units, sms * occ));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -545,37 +637,77 @@ cudaError_t launch_gemv_nt(const GemvParams<kGemvMaxLinears>& gp, int grid, size
   return cudaLaunchKernelEx(&cfg, kern, gp);
 }
 
-template <int NT>
-int occupancy_nt(size_t smem) {
-  int blocks = 0;
-  auto kern = gemv_streamk_kernel<NT, kGemvMaxLinears>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kGemvThreads, smem) != cudaSuccess)
-    return 1;
-  return blocks < 1 ? 1 : blocks;
+// Device tables of tensor maps for large launches, one per distinct list of
+// (planes address, N, K, r) and box width. Built with a synchronous copy the
+// first time a stack is served (so the first call must not be captured),
+// then reused by every later identical call.
+std::map<std::pair<int, std::vector<uint64_t>>, CUtensorMap*> g_map_tables;
+
+cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
+  int b0, b1;
+  plane_widths(j.r, b0, b1);
+  cudaError_t e = encode_map_2d(&out2[0], j.packed, uint64_t(j.N), uint64_t(j.K) * b0 / 8,
+                                static_cast<uint32_t>(P0), kRowsPerUnit, 1);
+  if (e != cudaSuccess || !b1) return e;
+  return encode_map_2d(&out2[1], j.packed + j.N * j.K * b0 / 8, uint64_t(j.N),
+                       uint64_t(j.K) * b1 / 8, static_cast<uint32_t>(P0 / 2), kRowsPerUnit, 1);
 }
 
-}  // namespace
+cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUtensorMap** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::vector<uint64_t> key;
+  key.reserve(size_t(n_jobs) * 4 + 1);
+  key.push_back(uint64_t(P0));
+  for (int i = 0; i < n_jobs; ++i) {
+    key.push_back(reinterpret_cast<uint64_t>(jobs[i].packed));
+    key.push_back(uint64_t(jobs[i].N));
+    key.push_back(uint64_t(jobs[i].K));
+    key.push_back(uint64_t(jobs[i].r));
+  }
+  std::lock_guard<std::mutex> lk(g_cache_mutex);
+  auto k2 = std::make_pair(dev, std::move(key));
+  auto it = g_map_tables.find(k2);
+  if (it != g_map_tables.end()) {
+    *out = it->second;
+    return cudaSuccess;
+  }
+  std::vector<CUtensorMap> host(size_t(n_jobs) * 2);
+  std::memset(host.data(), 0, host.size() * sizeof(CUtensorMap));
+  for (int i = 0; i < n_jobs; ++i) {
+    e = encode_plane_maps(jobs[i], P0, &host[size_t(2) * i]);
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap* dptr = nullptr;
+  e = cudaMalloc(&dptr, host.size() * sizeof(CUtensorMap));
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpy(dptr, host.data(), host.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) { cudaFree(dptr); return e; }
+  g_map_tables.emplace(std::move(k2), dptr);
+  *out = dptr;
+  return cudaSuccess;
+}
 
-cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream) {
-  if (n_jobs < 1 || n_jobs > kGemvMaxLinears || M < 1 || M > 32) return cudaErrorInvalidValue;
+template <int CAP>
+cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream) {
   // Bytes of low plane per row per unit: 192 keeps consecutive rows 64 bytes
   // apart modulo 128 (conflict-free 16-byte shared loads) with few copies;
   // larger batches use 64 to bound the staged activation block.
   const int P0 = M <= 8 ? 192 : 64;
   const int NT = (M + 7) / 8;
 
-  static thread_local GemvParams<kGemvMaxLinears> gp;
-  static thread_local PrepParams<kGemvMaxLinears> pp;
-  std::memset(&gp, 0, sizeof(gp));
-  std::memset(&pp, 0, sizeof(pp));
+  static thread_local GemvParams<CAP> gp;
+  static thread_local PrepParams<CAP> pp;
 
-  // Distinct inputs (class sums) and distinct (input, layout) pairs.
-  std::map<const void*, int> sum_of_x;
-  std::map<std::pair<const void*, int>, int> layout_of;
-  struct LayoutInfo { const void* x; int K, kc, w8, n_kc; size_t off; };
-  std::vector<LayoutInfo> layouts;
-  std::vector<std::pair<const void*, int>> sums;
+  // Distinct inputs (class sums) and distinct (input, layout) pairs. Few
+  // entries: linear scans are cheaper than maps here.
+  struct LayoutInfo { const void* x; int b0, K, kc, w8, n_kc; size_t off; };
+  LayoutInfo layouts[CAP];
+  const void* sum_x[CAP];
+  int sum_k[CAP];
+  int n_layouts = 0, n_sums = 0;
+  int lay_of[CAP], sum_of[CAP];
   bool two_planes = false;
   int units = 0;
   size_t xf_bytes = 0;
@@ -586,17 +718,18 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
     if (b1) two_planes = true;
     const int kc = P0 * 8 / b0;
     const int n_kc = static_cast<int>((j.K + kc - 1) / kc);
-    if (!sum_of_x.count(j.x)) {
-      sum_of_x[j.x] = static_cast<int>(sums.size());
-      sums.push_back({j.x, static_cast<int>(j.K)});
-    }
-    auto key = std::make_pair(j.x, b0);
-    if (!layout_of.count(key)) {
-      layout_of[key] = static_cast<int>(layouts.size());
-      layouts.push_back({j.x, static_cast<int>(j.K), kc, (128 / b0) / 8, n_kc, xf_bytes});
+    int si = 0;
+    while (si < n_sums && sum_x[si] != j.x) ++si;
+    if (si == n_sums) { sum_x[n_sums] = j.x; sum_k[n_sums] = static_cast<int>(j.K); ++n_sums; }
+    sum_of[i] = si;
+    int li = 0;
+    while (li < n_layouts && !(layouts[li].x == j.x && layouts[li].b0 == b0)) ++li;
+    if (li == n_layouts) {
+      layouts[n_layouts++] = {j.x, b0, static_cast<int>(j.K), kc, (128 / b0) / 8, n_kc, xf_bytes};
       xf_bytes += size_t(n_kc) * M * kc * 2;
       xf_bytes = (xf_bytes + 255) & ~size_t(255);
     }
+    lay_of[i] = li;
     const int nrb = static_cast<int>((j.N + kRowsPerUnit - 1) / kRowsPerUnit);
     LinDesc& d = gp.lin[i];
     d.plane0 = j.packed;
@@ -612,38 +745,46 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
     d.unit_begin = units;
     units += nrb * n_kc;
   }
+  if constexpr (CAP <= 8) {
+    for (int i = 0; i < n_jobs; ++i) {
+      cudaError_t em = encode_plane_maps(jobs[i], P0, &gp.maps[2 * i]);
+      if (em != cudaSuccess) return em;
+    }
+    gp.map_table = nullptr;
+  } else {
+    cudaError_t em = get_map_table(jobs, n_jobs, P0, &gp.map_table);
+    if (em != cudaSuccess) return em;
+  }
   const size_t psum_off = xf_bytes;
-  const size_t ws_bytes = psum_off + sums.size() * size_t(M) * 4 * sizeof(float) + 256;
+  const size_t ws_bytes = psum_off + size_t(n_sums) * M * 4 * sizeof(float) + 256;
   void* ws = nullptr;
   cudaError_t e = get_workspace(stream, ws_bytes, &ws);
   if (e != cudaSuccess) return e;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* psum_base = reinterpret_cast<float*>(wsb + psum_off);
   for (int i = 0; i < n_jobs; ++i) {
-    int b0, b1;
-    plane_widths(jobs[i].r, b0, b1);
-    gp.lin[i].xf = wsb + layouts[layout_of[std::make_pair(jobs[i].x, b0)]].off;
-    gp.lin[i].psum = psum_base + size_t(sum_of_x[jobs[i].x]) * M * 4;
+    gp.lin[i].xf = wsb + layouts[lay_of[i]].off;
+    gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * 4;
   }
 
   // Prep launch.
   pp.M = M;
-  pp.n_layout = static_cast<int>(layouts.size());
-  pp.n_sum = static_cast<int>(sums.size());
+  pp.n_layout = n_layouts;
+  pp.n_sum = n_sums;
   pp.n_zero = n_jobs;
-  for (size_t i = 0; i < layouts.size(); ++i) {
+  for (int i = 0; i < n_layouts; ++i) {
     pp.lay[i] = {static_cast<const __nv_bfloat16*>(layouts[i].x), wsb + layouts[i].off,
-                 layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc};
+                 layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc,
+                 layouts[i].b0 == 8 ? 1 : 0};
   }
-  for (size_t i = 0; i < sums.size(); ++i) {
-    pp.sum[i] = {static_cast<const __nv_bfloat16*>(sums[i].first), psum_base + i * M * 4,
-                 sums[i].second};
+  for (int i = 0; i < n_sums; ++i) {
+    pp.sum[i] = {static_cast<const __nv_bfloat16*>(sum_x[i]), psum_base + size_t(i) * M * 4, sum_k[i]};
   }
   for (int i = 0; i < n_jobs; ++i) pp.zero[i] = {jobs[i].y, int64_t(M) * jobs[i].N};
   const int sms = sm_count();
-  int prep_grid = std::max(pp.n_sum * M, sms);
+  int prep_grid = std::max(n_sums * M, sms);
   prep_grid = std::min(prep_grid, 4 * sms);
-  gemv_prep_kernel<kGemvMaxLinears><<<prep_grid, 256, 0, stream>>>(pp);
+  gemv_prep_kernel<CAP><<<prep_grid, 256, 0, stream>>>(pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -654,8 +795,7 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
   const uint32_t x_bytes = static_cast<uint32_t>(M * (P0 * 8 / 2) * 2);  // largest KC (b0 = 2)
   uint32_t stage_bytes = off_x + x_bytes;
   stage_bytes = (stage_bytes + 127) & ~127u;
-  const size_t budget = 110 * 1024;
-  int stages = static_cast<int>(budget / stage_bytes);
+  int stages = static_cast<int>(kStageBudget / stage_bytes);
   stages = std::max(2, std::min(stages, kMaxStages));
   const size_t smem = kBarrierBytes + size_t(stages) * stage_bytes;
 
@@ -674,20 +814,21 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
   gp.err = err;
   gp.wait_ns = wait_limit_ns();
 
-  int occ = 1;
   switch (NT) {
-    case 1: occ = occupancy_nt<1>(smem); break;
-    case 2: occ = occupancy_nt<2>(smem); break;
-    case 3: occ = occupancy_nt<3>(smem); break;
-    default: occ = occupancy_nt<4>(smem); break;
+    case 1: return launch_gemv<1, CAP>(gp, smem, sms, units, stream);
+    case 2: return launch_gemv<2, CAP>(gp, smem, sms, units, stream);
+    case 3: return launch_gemv<3, CAP>(gp, smem, sms, units, stream);
+    default: return launch_gemv<4, CAP>(gp, smem, sms, units, stream);
   }
-  const int grid = std::max(1, std::min(units, sms * occ));
-  switch (NT) {
-    case 1: return launch_gemv_nt<1>(gp, grid, smem, stream);
-    case 2: return launch_gemv_nt<2>(gp, grid, smem, stream);
-    case 3: return launch_gemv_nt<3>(gp, grid, smem, stream);
-    default: return launch_gemv_nt<4>(gp, grid, smem, stream);
-  }
+}
+
+}  // namespace
+
+cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream) {
+  if (n_jobs < 1 || n_jobs > kGemvMaxLinears || M < 1 || M > 32) return cudaErrorInvalidValue;
+  if (n_jobs == 1) return run_gemv_cap<1>(jobs, n_jobs, M, stream);
+  if (n_jobs <= 8) return run_gemv_cap<8>(jobs, n_jobs, M, stream);
+  return run_gemv_cap<kGemvMaxLinears>(jobs, n_jobs, M, stream);
 }
 
 }  // namespace mq

@@ -1,6 +1,7 @@
 // Host-side declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -43,6 +44,12 @@ cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out);
 // Device error word of the current device (zero-initialized).
 cudaError_t get_error_word(uint32_t** out);
 uint64_t wait_limit_ns();
+
+// 2-D tensor map over a row-major matrix of `rows` x `row_elems` elements of
+// `elem_bytes` bytes (1: uint8, 2: bf16), box `box_inner` x `box_rows`, no
+// swizzle, out-of-bounds elements read as zero. Cached per arguments.
+cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t row_elems,
+                          uint32_t box_inner, uint32_t box_rows, int elem_bytes);
 int sm_count();
 
 cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
