@@ -1,0 +1,524 @@
+"""Benchmark of the nested-bit int8 serving path on B200.
+
+Headline workload: the Mix'n'Match 7B-shaped decode stack -- 32 layers x
+(qkv 6144x4096, o 4096x4096, gate 14336x4096, up 14336x4096,
+down 4096x14336), widths int8 on the first/last 4 layers, int4 on the next
+4 inward, int2 on layers 8..23 -- streamed once per token (M = 1) through
+mq_stack_forward. One step = one forward of every linear of the stack.
+Metric: sliced-int GEMV effective HBM GB/s (packed-weight bytes / step
+time), with % of the measured HBM peak and us/layer at r = 8, 4, 2.
+
+The other parts of the path (int8 container quantize, slice-pack, a single
+decode linear, the prefill GEMM) are timed separately and reported under
+"rows".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--M 1]
+       python bench.py --impl reference ...   (CPU oracle arm)
+For N > 1 launch under torch.distributed.run: every rank serves its own
+replica of the stack (no data-path collective), value = sum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+import synth
+
+WORKLOAD = "mixnmatch_7b_stack"
+METRIC = "sliced-int GEMV effective HBM GB/s (% of peak) and us/layer at r=8/4/2"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1606.7)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        import tempfile
+        self.path = tempfile.mktemp(prefix="mq_clocks_", suffix=".csv")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=self.fh, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)  # let the sampler start before the timed region
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        with open(self.path) as f:
+            self.lines = [ln.strip() for ln in f]
+        os.unlink(self.path)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    """Returns (rank, world, local_rank). Uses torch.distributed when launched
+    by torch.distributed.run (WORLD_SIZE > 1)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def dist_max(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- GPU arm
+class Stack:
+    """The packed 7B Mix'n'Match stack resident in HBM."""
+
+    def __init__(self, M: int, dev, layers: int = 32, seed_base: int = 1000):
+        import torch
+        import nested_bit_weight_int8_b200 as mq
+        self.mq, self.torch, self.dev, self.M = mq, torch, dev, M
+        self.widths = synth.mixnmatch_widths(layers)
+        mats = synth.WORKLOADS[WORKLOAD]["mats"]
+        self.Ks = sorted({k for _, _, k in mats})
+        gen = torch.Generator(device=dev)
+        self.x = {}
+        for k in self.Ks:
+            gen.manual_seed(2000 + M + k)
+            self.x[k] = torch.randn((M, k), generator=gen, device=dev).to(torch.bfloat16)
+        self.lins, self.lol, self.bytes_by_width, self.layer_of = [], [], {}, []
+        self.packed_bytes = 0
+        self.rows_total = 0
+        # all outputs live in one buffer so the result leaves the device in one copy
+        n_out = sum(n for _, n, _ in mats) * layers
+        self.y_all = torch.empty(M * n_out, dtype=torch.float32, device=dev)
+        y_off = 0
+        for layer in range(layers):
+            r = self.widths[layer]
+            for j, (_, n, k) in enumerate(mats):
+                gen.manual_seed(seed_base + 5 * layer + j)
+                w = (torch.randn((n, k), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+                q = torch.empty((n, k), dtype=torch.uint8, device=dev)
+                a = torch.empty(n, dtype=torch.float32, device=dev)
+                z = torch.empty(n, dtype=torch.float32, device=dev)
+                mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z)
+                p = torch.empty(mq.packed_bytes(n, k, r), dtype=torch.uint8, device=dev)
+                mq.slice_pack(q, n, k, r, p)
+                del w, q
+                y = self.y_all[y_off:y_off + M * n].view(M, n)
+                y_off += M * n
+                self.lins.append((self.x[k], p, a, z, y, n, k))
+                self.lol.append(layer)
+                nb = n * k * r // 8
+                self.packed_bytes += nb
+                self.bytes_by_width[r] = self.bytes_by_width.get(r, 0) + nb
+                self.rows_total += n
+        self.layers = layers
+        torch.cuda.synchronize()
+
+    def step(self, stream=None):
+        self.mq.stack_forward(self.lins, self.lol, self.widths, self.M, stream)
+
+    def sub_stack(self, width: int):
+        """The linears of the layers at one width, as their own stack."""
+        idx = [i for i, l in enumerate(self.lol) if self.widths[l] == width]
+        layers = sorted({self.lol[i] for i in idx})
+        remap = {l: j for j, l in enumerate(layers)}
+        lins = [self.lins[i] for i in idx]
+        lol = [remap[self.lol[i]] for i in idx]
+        return lins, lol, [width] * len(layers), len(layers)
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes the step must move: packed planes + alpha, z + x + y."""
+        xb = sum(2 * self.M * k for (_, _, _, _, _, n, k) in self.lins)
+        yb = sum(4 * self.M * n for (_, _, _, _, _, n, k) in self.lins)
+        return self.packed_bytes + 8 * self.rows_total + xb + yb
+
+
+def time_device(fn, steps: int, warmup: int, stream, world: int, dev):
+    """CUDA-event time of `steps` calls of fn on `stream`, barrier and
+    synchronize on both sides, max over ranks. Returns ms per step."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist_barrier(world, dev)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world, dev)
+    ms = e0.elapsed_time(e1) / steps
+    return dist_max(ms, world, dev)
+
+
+def rows_timings(dev, stream):
+    """Separately timed rows of the path on one 14336x4096 bf16 weight:
+    quantize (Eq. 1), slice-pack (Eq. 6) per width, one decode linear per
+    width (M = 1), and the prefill GEMM at M = 2048 when served."""
+    import torch
+    import nested_bit_weight_int8_b200 as mq
+    n, k = 14336, 4096
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(300)
+    w = (torch.randn((n, k), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    q = torch.empty((n, k), dtype=torch.uint8, device=dev)
+    a = torch.empty(n, dtype=torch.float32, device=dev)
+    z = torch.empty(n, dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def timed(fn, reps=10):
+        fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps * 1000.0  # us
+
+    out = {}
+    us = timed(lambda: mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z, stream))
+    out["quantize_int8_14336x4096"] = {"us": round(us, 2), "GBps": round((n * k * 3 + 8 * n) / us / 1e3, 1)}
+    x = torch.randn((1, k), generator=gen, device=dev).to(torch.bfloat16)
+    y = torch.empty((1, n), dtype=torch.float32, device=dev)
+    for r in (8, 4, 2):
+        p = torch.empty(mq.packed_bytes(n, k, r), dtype=torch.uint8, device=dev)
+        us = timed(lambda: mq.slice_pack(q, n, k, r, p, stream))
+        out[f"slice_pack_r{r}"] = {"us": round(us, 2), "GBps": round((n * k + n * k * r // 8) / us / 1e3, 1)}
+        us = timed(lambda: mq.linear(x, 1, k, p, a, z, n, r, y, stream))
+        out[f"decode_linear_r{r}_M1"] = {"us": round(us, 2), "GBps": round(n * k * r / 8 / us / 1e3, 1)}
+    try:
+        m = 2048
+        xm = torch.randn((m, k), generator=gen, device=dev).to(torch.bfloat16)
+        ym = torch.empty((m, n), dtype=torch.float32, device=dev)
+        p = torch.empty(mq.packed_bytes(n, k, 4), dtype=torch.uint8, device=dev)
+        mq.slice_pack(q, n, k, 4, p, stream)
+        us = timed(lambda: mq.linear(xm, m, k, p, a, z, n, 4, ym, stream), reps=5)
+        out["prefill_gemm_r4_M2048"] = {"us": round(us, 2), "TFLOPs": round(2 * m * n * k / us / 1e6, 1)}
+    except mq.MQError as e:
+        out["prefill_gemm_r4_M2048"] = {"unavailable": str(e)}
+    torch.cuda.synchronize()
+    return out
+
+
+def cpu_baseline(M: int, budget_s: float = 12.0):
+    """The CPU oracle (float64 numpy) on a bounded sample of the same
+    workload: dequantize-and-multiply for row blocks of the stack's linears,
+    repeated until about budget_s seconds of CPU work. Returns the same
+    metric (effective packed-weight GB/s) and what the sample was."""
+    import oracle
+    widths = synth.mixnmatch_widths(32)
+    shapes = synth.stack_shapes(32)
+    rows = 512
+    done_bytes, t_used, n_blocks = 0, 0.0, 0
+    picks = [0, 5 * 4 + 2, 5 * 12 + 4, 5 * 16 + 1, 5 * 31 + 3]  # linears at r = 8, 4, 2, 2, 8
+    i = 0
+    while t_used < budget_s and i < 400:
+        layer, name, n, k, seed = shapes[picks[i % len(picks)]]
+        r = widths[layer]
+        w = synth.f32_from_bf16_bits(synth.gaussian_weights(rows, k, seed + 7919 * i)).astype(np.float64)
+        x = synth.f32_from_bf16_bits(synth.activations(M, k, 2000 + M + k)).astype(np.float64)
+        q, a, z = oracle.quantize_minmax(w)
+        t0 = time.perf_counter()
+        y = oracle.linear(x, oracle.dequant_slice(q, a, z, r))
+        t_used += time.perf_counter() - t0
+        done_bytes += rows * k * r // 8
+        n_blocks += 1
+        i += 1
+        del y
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    return {"value": round(done_bytes / t_used / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n_blocks} blocks of {rows} rows from stack linears at their widths "
+                      f"(dequantize + float64 matmul per block, M={M}), {t_used:.1f}s of CPU work"}
+
+
+def run_gpu(args, rank, world, local):
+    import torch
+    import nested_bit_weight_int8_b200 as mq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    hbm_peak, bf16_peak, peak_kind = _peaks()
+    with torch.cuda.stream(stream):
+        stack = Stack(args.M, dev)
+        stack.step(stream)
+        torch.cuda.synchronize()
+        mq.device_status(stream)
+        launches_per_step = 2 * ((len(stack.lins) + 255) // 256)
+
+        clocks = ClockSampler(local)
+        clocks.start()
+        ms = time_device(lambda: stack.step(stream), args.steps, args.warmup, stream, world, dev)
+        clk = clocks.stop()
+        mq.device_status(stream)
+
+        # us/layer at each width: the layers of one width as their own stack
+        per_width = {}
+        for r in (8, 4, 2):
+            lins, lol, wd, nl = stack.sub_stack(r)
+            msr = time_device(lambda: mq.stack_forward(lins, lol, wd, args.M, stream),
+                              max(3, args.steps // 4), 3, stream, world, dev)
+            per_width[f"r{r}"] = {"layers": nl, "us_per_layer": round(msr * 1000 / nl, 2),
+                                  "GBps": round(stack.bytes_by_width[r] / (msr * 1e-3) / 1e9, 1)}
+
+        # end to end through the C ABI with host buffers: pinned x in, y out
+        xs_host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in stack.x.items()}
+        for k, v in xs_host.items():
+            v.copy_(stack.x[k].cpu())
+        y_host = torch.empty(stack.y_all.shape, dtype=torch.float32, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for v in xs_host.values())
+        d2h = y_host.numel() * 4
+
+        def e2e_step():
+            for k, v in xs_host.items():
+                stack.x[k].copy_(v, non_blocking=True)
+            stack.step(stream)
+            y_host.copy_(stack.y_all, non_blocking=True)
+
+        ms_e2e = time_device(e2e_step, max(3, args.steps // 4), 3, stream, world, dev)
+
+        rows = rows_timings(dev, stream) if rank == 0 and not args.no_rows else {}
+    torch.cuda.synchronize()
+
+    gbs = stack.packed_bytes / (ms * 1e-3) / 1e9
+    algo = stack.algorithmic_bytes()
+    achieved = algo / (ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(gbs * world, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 x int-code planes, fp32 accumulate",
+        "data": "synthetic (seeded torch normal weights N(0,0.02^2), activations N(0,1))",
+        "config": {
+            "workload": WORKLOAD,
+            "layers": stack.layers,
+            "widths": "int8 x8 (layers 0-3, 28-31), int4 x8 (4-7, 24-27), int2 x16 (8-23)",
+            "M": args.M,
+            "linears": len(stack.lins),
+            "packed_bytes_per_step": stack.packed_bytes,
+            "l2": "inputs larger than L2: 3.49 GB of packed planes streamed per step",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "pct_of_hbm_peak": round(100 * gbs / hbm_peak, 1),
+        "us_per_layer": round(ms * 1000 / stack.layers, 2),
+        "tokens_per_s": round(args.M * world * 1000.0 / ms, 1),
+        "per_width": per_width,
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": None,
+            "peak_kind": peak_kind,
+            "kernel": "gemv_streamk_kernel (timed with its prep kernel, one step)",
+        },
+        "e2e": {
+            "value": round(stack.packed_bytes / (ms_e2e * 1e-3) / 1e9 * world, 1),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms_e2e, 4),
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "rows": rows,
+    }
+    tr = _profile_traffic()
+    if tr is not None and tr.get("kernel_source_hash") == _kernel_hash():
+        out["roofline"]["traffic"] = tr.get("dram_bytes_per_launch")
+    return out
+
+
+def _profile_traffic():
+    """DRAM bytes per launch of the stack kernel from the committed ncu
+    summary (lines "key: value"), or None."""
+    path = os.path.join(ROOT, "profiles", "gemv_streamk_mixnmatch_7b_M1.md")
+    if not os.path.exists(path):
+        return None
+    d = {}
+    with open(path) as f:
+        for ln in f:
+            if ":" in ln and not ln.startswith("#"):
+                k, v = ln.split(":", 1)
+                d[k.strip().strip("-* `")] = v.strip().strip("`")
+    try:
+        return {"dram_bytes_per_launch": float(d["dram_bytes_per_launch"]),
+                "kernel_source_hash": d["kernel_source_hash"]}
+    except (KeyError, ValueError):
+        return None
+
+
+def _kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nested_bit_weight_int8_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_reference(args, rank, world):
+    """CPU oracle arm: the float64 oracle on the host cores, each step a
+    bounded sample of the same workload, same metric and unit."""
+    budget = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(args.M, budget_s=budget / 4)
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(args.M, budget_s=budget))
+    v = float(np.median([b["value"] for b in vals]))
+    last = vals[-1]
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(v, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": None,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": WORKLOAD, "M": args.M, "sample": last["sample"]},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        # the CPU oracle arm: rank 0 alone runs and prints; other ranks exit
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps(run_reference(args, 0, world)), flush=True)
+        return 0
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        out = run_gpu(args, rank, world, local)
+        if rank == 0:
+            if not args.no_cpu:
+                out["cpu_baseline"] = cpu_baseline(args.M)
+            print(json.dumps(out), flush=True)
+        return 0
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
