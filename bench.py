@@ -152,11 +152,12 @@ def dist_done(world: int):
 class Stack:
     """The packed 7B Mix'n'Match stack resident in HBM."""
 
-    def __init__(self, M: int, dev, layers: int = 32, seed_base: int = 1000):
+    def __init__(self, M: int, dev, layers: int = 32, seed_base: int = 1000, widths=None):
         import torch
         import nested_bit_weight_int8_b200 as mq
         self.mq, self.torch, self.dev, self.M = mq, torch, dev, M
-        self.widths = synth.mixnmatch_widths(layers)
+        self.widths = list(widths) if widths else synth.mixnmatch_widths(layers)
+        layers = len(self.widths)
         mats = synth.WORKLOADS[WORKLOAD]["mats"]
         self.Ks = sorted({k for _, _, k in mats})
         gen = torch.Generator(device=dev)
@@ -179,9 +180,10 @@ class Stack:
                 q = torch.empty((n, k), dtype=torch.uint8, device=dev)
                 a = torch.empty(n, dtype=torch.float32, device=dev)
                 z = torch.empty(n, dtype=torch.float32, device=dev)
-                mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z)
+                cur = torch.cuda.current_stream(dev)
+                mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z, cur)
                 p = torch.empty(mq.packed_bytes(n, k, r), dtype=torch.uint8, device=dev)
-                mq.slice_pack(q, n, k, r, p)
+                mq.slice_pack(q, n, k, r, p, cur)
                 del w, q
                 y = self.y_all[y_off:y_off + M * n].view(M, n)
                 y_off += M * n
@@ -332,7 +334,8 @@ def run_gpu(args, rank, world, local):
     stream = torch.cuda.Stream(device=dev)
     hbm_peak, bf16_peak, peak_kind = _peaks()
     with torch.cuda.stream(stream):
-        stack = Stack(args.M, dev)
+        widths = [int(v) for v in args.widths.split(",")] if args.widths else None
+        stack = Stack(args.M, dev, layers=args.layers, widths=widths)
         stack.step(stream)
         torch.cuda.synchronize()
         mq.device_status(stream)
@@ -346,7 +349,7 @@ def run_gpu(args, rank, world, local):
 
         # us/layer at each width: the layers of one width as their own stack
         per_width = {}
-        for r in (8, 4, 2):
+        for r in sorted(set(stack.widths), reverse=True):
             lins, lol, wd, nl = stack.sub_stack(r)
             msr = time_device(lambda: mq.stack_forward(lins, lol, wd, args.M, stream),
                               max(3, args.steps // 4), 3, stream, world, dev)
@@ -391,7 +394,8 @@ def run_gpu(args, rank, world, local):
         "config": {
             "workload": WORKLOAD,
             "layers": stack.layers,
-            "widths": "int8 x8 (layers 0-3, 28-31), int4 x8 (4-7, 24-27), int2 x16 (8-23)",
+            "widths": ("int8 x8 (layers 0-3, 28-31), int4 x8 (4-7, 24-27), int2 x16 (8-23)"
+                       if stack.widths == synth.mixnmatch_widths(32) else stack.widths),
             "M": args.M,
             "linears": len(stack.lins),
             "packed_bytes_per_step": stack.packed_bytes,
@@ -496,6 +500,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--layers", type=int, default=32,
+                    help="layers of the 7B-shaped stack (widths follow the Mix'n'Match pattern)")
+    ap.add_argument("--widths", default="",
+                    help="comma-separated per-layer widths; overrides --layers (small profiling stacks)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmq.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m nested_bit_weight_int8_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python nested_bit_weight_int8_b200/build.py` "
         "(nvcc, sm_100a). There is no fallback implementation.")
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -402,12 +402,13 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         issue_x(c, s);
         cursor_next(p, c);
       }
-      if (aborted) {
-        // Leave no bulk copy in flight: wait for the last issue of every stage.
-        const int first = issued > S ? issued - S : 0;
-        for (int j = first; j < issued; ++j) {
-          if (!mbar_wait_bounded(&full[j % S], (j / S) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
-        }
+      // Leave no bulk copy in flight when this thread exits, whether or not
+      // the consumers took the data (they stop early after a wait gave up):
+      // wait for the last issue of every stage.
+      (void)aborted;
+      const int first = issued > S ? issued - S : 0;
+      for (int j = first; j < issued; ++j) {
+        if (!mbar_wait_bounded(&full[j % S], (j / S) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
       }
     } else {
       pdl_wait_primary();
