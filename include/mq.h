@@ -150,6 +150,47 @@ MQ_API mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_o
                            int n_lins, const int* widths, int n_layers,
                            int64_t M, void* stream);
 
+/* Bytes of the device array that mq_linear_noalloc works in (1.25 MiB). */
+#define MQ_NOALLOC_SCRATCH_BYTES (1280u * 1024u)
+
+/*
+ * mq_linear_noalloc -- the decode GEMV of mq_linear (1 <= M <= 32) without any
+ * device allocation. The paper has no counterpart: this is a deployment aid.
+ *
+ * Who needs it: callers that may not, or cannot afford to, call cudaMalloc. For
+ * example, a serving engine whose own allocator owns every byte of HBM. Or a
+ * plugin loaded into a host program that forbids it to allocate. Or a
+ * latency-critical decode loop where an allocation, and the device-wide
+ * synchronization it can imply, is not acceptable. mq_linear would allocate
+ * its per-stream workspace and error word on first use; this entry point
+ * does not.
+ *
+ * Instead its scratch lives in one file-scope device array of
+ * MQ_NOALLOC_SCRATCH_BYTES. The first 256 bytes hold a wait-error word; the
+ * rest holds the fragment-ordered activation blocks and activation sums.
+ * Every GPU that loads the library holds this array until the process exits.
+ * It is enough for M * K up to 524288 (e.g. M = 32 with K = 16384). A call
+ * that needs more returns MQ_ERR_INVALID_ARG with the sizes in
+ * mq_last_error() and launches nothing.
+ *
+ * Arguments, layouts and accuracy: as mq_linear, with 1 <= M <= 32.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the array's device address and zeroes its error word with a synchronous
+ * cudaMemset plus a device synchronization. Make that first call before any
+ * stream capture.
+ *
+ * Sharing: every call uses the same array, and the array keeps what the last
+ * call wrote. Each call rewrites on the device all the scratch it reads, and
+ * zeroes y there before accumulating. Calls whose kernels overlap on the GPU race: two streams,
+ * or two host threads on one device. Serialize them. A bounded wait that gave
+ * up leaves y undefined. It is recorded in the array's error word, not in the
+ * word that mq_device_status() reads.
+ */
+MQ_API mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, const void* packed,
+                                   const float* alpha, const float* zero, int64_t N, int r,
+                                   float* y, void* stream);
+
 /*
  * Synchronizes `stream`, then reports whether any kernel launched by this
  * library on the current device gave up a bounded wait (MQ_ERR_TIMEOUT; the

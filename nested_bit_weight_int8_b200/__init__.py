@@ -52,13 +52,17 @@ _linear = _sig("mq_linear", _int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _
 _stack = _sig("mq_stack_forward", _int,
               [ctypes.POINTER(LinearDesc), ctypes.POINTER(_int), _int, ctypes.POINTER(_int), _int,
                _i64, _vp])
+_linear_noalloc = _sig("mq_linear_noalloc", _int,
+                      [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
 _device_status = _sig("mq_device_status", _int, [_vp])
 _release = _sig("mq_release_workspace", _int, [])
 _wait_limit = _sig("mq_debug_set_wait_limit_ns", _int, [_u64])
 
 EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8",
             "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
-            "mq_release_workspace", "mq_debug_set_wait_limit_ns")
+            "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc")
+
+NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
 
 class MQError(RuntimeError):
@@ -116,6 +120,14 @@ def linear(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=Non
                    _stream(stream)))
 
 
+def linear_noalloc(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=None) -> None:
+    """As linear() for 1 <= M <= 32, but working in the library's fixed device
+    array instead of allocating a workspace (for callers that cannot allocate).
+    Calls that overlap on the GPU share that array and race."""
+    _check(_linear_noalloc(_ptr(x), M, K, _ptr(packed), _ptr(alpha), _ptr(zero), N, r, _ptr(y),
+                           _stream(stream)))
+
+
 def stack_forward(lins, layer_of_lin, widths, M: int, stream=None) -> None:
     """Mix'n'Match stack. lins: sequence of (x, packed, alpha, zero, y, N, K)."""
     n = len(lins)
@@ -144,4 +156,4 @@ def raw_status(fn_name: str, *args) -> int:
     """Calls a C entry point and returns its status code without raising
     (used by tests of the argument checks)."""
     return {"mq_quantize_int8": _quantize, "mq_slice_pack": _slice_pack,
-            "mq_linear": _linear}[fn_name](*args)
+            "mq_linear": _linear, "mq_linear_noalloc": _linear_noalloc}[fn_name](*args)

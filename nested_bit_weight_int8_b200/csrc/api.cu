@@ -100,6 +100,8 @@ cudaError_t get_error_word(uint32_t** out) {
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 }  // namespace mq
 
 using namespace mq;

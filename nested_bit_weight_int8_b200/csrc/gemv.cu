@@ -691,7 +691,8 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
 }
 
 template <int CAP>
-cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream) {
+cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream,
+                         const FixedScratch* fixed = nullptr) {
   // Bytes of low plane per row per unit: 192 keeps consecutive rows 64 bytes
   // apart modulo 128 (conflict-free 16-byte shared loads) with few copies;
   // larger batches use 64 to bound the staged activation block.
@@ -759,8 +760,14 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   const size_t psum_off = xf_bytes;
   const size_t ws_bytes = psum_off + size_t(n_sums) * M * 4 * sizeof(float) + 256;
   void* ws = nullptr;
-  cudaError_t e = get_workspace(stream, ws_bytes, &ws);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (fixed) {
+    if (ws_bytes > fixed->bytes) return cudaErrorMemoryAllocation;
+    ws = fixed->ptr;
+  } else {
+    e = get_workspace(stream, ws_bytes, &ws);
+    if (e != cudaSuccess) return e;
+  }
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* psum_base = reinterpret_cast<float*>(wsb + psum_off);
   for (int i = 0; i < n_jobs; ++i) {
@@ -810,8 +817,12 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.pitch0 = P0;
   gp.pitch1 = P1;
   uint32_t* err = nullptr;
-  e = get_error_word(&err);
-  if (e != cudaSuccess) return e;
+  if (fixed) {
+    err = fixed->err;
+  } else {
+    e = get_error_word(&err);
+    if (e != cudaSuccess) return e;
+  }
   gp.err = err;
   gp.wait_ns = wait_limit_ns();
 
@@ -830,6 +841,24 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
   if (n_jobs == 1) return run_gemv_cap<1>(jobs, n_jobs, M, stream);
   if (n_jobs <= 8) return run_gemv_cap<8>(jobs, n_jobs, M, stream);
   return run_gemv_cap<kGemvMaxLinears>(jobs, n_jobs, M, stream);
+}
+
+size_t gemv_scratch_bytes(const LinearJob& job, int M) {
+  // Same arithmetic as the planner in run_gemv_cap for one linear.
+  const int P0 = M <= 8 ? 192 : 64;
+  int b0, b1;
+  plane_widths(job.r, b0, b1);
+  const int kc = P0 * 8 / b0;
+  const int64_t n_kc = (job.K + kc - 1) / kc;
+  size_t xf = size_t(n_kc) * M * kc * 2;
+  xf = (xf + 255) & ~size_t(255);
+  return xf + size_t(M) * 4 * sizeof(float) + 256;
+}
+
+cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
+                           const FixedScratch& scratch) {
+  if (M < 1 || M > 32) return cudaErrorInvalidValue;
+  return run_gemv_cap<1>(&job, 1, M, stream, &scratch);
 }
 
 }  // namespace mq

@@ -44,6 +44,8 @@ cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out);
 // Device error word of the current device (zero-initialized).
 cudaError_t get_error_word(uint32_t** out);
 uint64_t wait_limit_ns();
+// Replaces the calling thread's mq_last_error() text.
+void set_last_error(const char* msg);
 
 // 2-D tensor map over a row-major matrix of `rows` x `row_elems` elements of
 // `elem_bytes` bytes (1: uint8, 2: bf16), box `box_inner` x `box_rows`, no
@@ -61,6 +63,21 @@ cudaError_t launch_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, voi
 // persistent stream-K GEMV over all jobs (at most kGemvMaxLinears).
 constexpr int kGemvMaxLinears = 256;
 cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream);
+
+// Caller-provided device scratch for the decode path: `ptr` (256-byte
+// aligned, `bytes` long) replaces the per-stream workspace and `err` the
+// per-device error word. Used by the entry point that allocates nothing.
+struct FixedScratch {
+  void* ptr;
+  size_t bytes;
+  uint32_t* err;
+};
+// Scratch bytes the decode path needs for one linear at batch M.
+size_t gemv_scratch_bytes(const LinearJob& job, int M);
+// Decode path for one linear on caller-provided scratch; returns
+// cudaErrorMemoryAllocation if the scratch is too small (nothing launched).
+cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
+                           const FixedScratch& scratch);
 
 // Prefill path (M > 32): tcgen05 GEMM for one linear.
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);

@@ -1,0 +1,69 @@
+"""mq_linear_noalloc: the decode GEMV for callers that cannot allocate device
+memory (an engine whose allocator owns all of HBM, a plugin that may not
+allocate, a decode loop that cannot afford an allocation's synchronization).
+
+It must give the same results as mq_linear, within the tolerance every parity
+test here uses (|dy| <= 1e-3 sum_k |x||W_r| + 1e-6), on consecutive calls that
+share its one fixed device array. This file is named so that pytest collects it
+last.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nested_bit_weight_int8_b200 as mq
+import oracle
+import synth
+
+
+def _tolerance(x_bits, q, a, z, r):
+    x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
+    return oracle.tolerance(x_vals, oracle.dequant_slice(q, a, z, r))
+
+
+def test_noalloc_rejects_oversized_calls_on_the_host():
+    """Sizes beyond the fixed array are refused before any CUDA call."""
+    F = 1 << 20
+    st = mq.raw_status("mq_linear_noalloc", F, 32, 32768, F, F, F, 64, 4, F, None)
+    assert st == mq.MQ_ERR_INVALID_ARG
+    assert "scratch" in mq.last_error()
+    assert mq.raw_status("mq_linear_noalloc", F, 33, 256, F, F, F, 64, 4, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_linear_noalloc", F, 1, 256, F, F, F, 64, 5, F, None) == mq.MQ_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_linear_on_consecutive_calls():
+    dev = "cuda:0"
+    torch.cuda.set_device(0)
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+
+    # (M, N, K, r, weight seed): the second call is the largest M * K the
+    # fixed array serves, with another width and shape, so it reuses the
+    # array after the first call left its own contents there.
+    cases = [(8, 2048, 4096, 4, 31), (32, 1000, 16384, 2, 32), (1, 777, 2304, 8, 33)]
+    for M, N, K, r, seed in cases:
+        w = synth.f32_from_bf16_bits(synth.gaussian_weights(N, K, seed)).astype(np.float64)
+        q, a, z = oracle.quantize_minmax(w)
+        x_bits = synth.activations(M, K, seed + 100)
+        x, a_d, z_d = up(x_bits), up(a), up(z)
+        packed = torch.empty(mq.packed_bytes(N, K, r), dtype=torch.uint8, device=dev)
+        mq.slice_pack(up(q), N, K, r, packed)
+
+        y_lin = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        mq.linear(x, M, K, packed, a_d, z_d, N, r, y_lin)
+        y_na = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        mq.linear_noalloc(x, M, K, packed, a_d, z_d, N, r, y_na)
+        torch.cuda.synchronize()
+        mq.device_status()
+
+        y1 = y_lin.cpu().numpy().astype(np.float64)
+        y2 = y_na.cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(y2)), f"M={M} N={N} K={K} r={r}: unwritten output"
+        tol = _tolerance(x_bits, q, a, z, r)
+        err = np.abs(y2 - y1)
+        assert np.all(err <= tol), (
+            f"M={M} N={N} K={K} r={r}: {int((err > tol).sum())} elements differ from mq_linear "
+            f"beyond the tolerance (max ratio {float((err / tol).max()):.3g})")
