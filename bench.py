@@ -197,7 +197,9 @@ class Stack:
         torch.cuda.synchronize()
 
     def step(self, stream=None):
-        self.mq.stack_forward(self.lins, self.lol, self.widths, self.M, stream)
+        if getattr(self, "_plan", None) is None:
+            self._plan = self.mq.StackPlan(self.lins, self.lol, self.widths, self.M)
+        self._plan.run(stream)
 
     def sub_stack(self, width: int):
         """The linears of the layers at one width, as their own stack."""
@@ -351,7 +353,8 @@ def run_gpu(args, rank, world, local):
         per_width = {}
         for r in sorted(set(stack.widths), reverse=True):
             lins, lol, wd, nl = stack.sub_stack(r)
-            msr = time_device(lambda: mq.stack_forward(lins, lol, wd, args.M, stream),
+            plan = mq.StackPlan(lins, lol, wd, args.M)
+            msr = time_device(lambda: plan.run(stream),
                               max(3, args.steps // 4), 3, stream, world, dev)
             per_width[f"r{r}"] = {"layers": nl, "us_per_layer": round(msr * 1000 / nl, 2),
                                   "GBps": round(stack.bytes_by_width[r] / (msr * 1e-3) / 1e9, 1)}

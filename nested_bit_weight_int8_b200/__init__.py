@@ -128,15 +128,32 @@ def linear_noalloc(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, st
                            _stream(stream)))
 
 
+class StackPlan:
+    """The arguments of one Mix'n'Match stack call, marshalled once.
+
+    lins: sequence of (x, packed, alpha, zero, y, N, K); layer_of_lin[i] is
+    the layer of linear i and widths[layer] its width. run() then makes the
+    same mq_stack_forward call without rebuilding the descriptor arrays.
+    The tensors must stay alive (the plan keeps references to them).
+    """
+
+    def __init__(self, lins, layer_of_lin, widths, M: int):
+        n = len(lins)
+        self._keep = list(lins)
+        self._arr = (LinearDesc * n)()
+        for i, (x, packed, alpha, zero, y, N, K) in enumerate(lins):
+            self._arr[i] = LinearDesc(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(zero), _ptr(y), N, K)
+        self._lol = (_int * n)(*layer_of_lin)
+        self._wd = (_int * len(widths))(*widths)
+        self._n, self._nl, self._M = n, len(widths), M
+
+    def run(self, stream=None) -> None:
+        _check(_stack(self._arr, self._lol, self._n, self._wd, self._nl, self._M, _stream(stream)))
+
+
 def stack_forward(lins, layer_of_lin, widths, M: int, stream=None) -> None:
     """Mix'n'Match stack. lins: sequence of (x, packed, alpha, zero, y, N, K)."""
-    n = len(lins)
-    arr = (LinearDesc * n)()
-    for i, (x, packed, alpha, zero, y, N, K) in enumerate(lins):
-        arr[i] = LinearDesc(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(zero), _ptr(y), N, K)
-    lol = (_int * n)(*layer_of_lin)
-    wd = (_int * len(widths))(*widths)
-    _check(_stack(arr, lol, n, wd, len(widths), M, _stream(stream)))
+    StackPlan(lins, layer_of_lin, widths, M).run(stream)
 
 
 def device_status(stream=None) -> None:

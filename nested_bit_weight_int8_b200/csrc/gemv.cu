@@ -5,9 +5,13 @@
 //
 // Work decomposition. A "unit" is 128 weight rows x KC codes of one linear.
 // All units of all linears of a launch form one list; CTA c of a persistent
-// grid of G CTAs takes the contiguous range [c*U/G, (c+1)*U/G) ("stream-K"),
-// so every CTA streams the same number of units whatever the shapes. Partial
-// row sums are added into y with fp32 atomics; the prep kernel zeroes y.
+// grid of G CTAs takes a contiguous range of it ("stream-K"). The ranges are
+// cut on the host so that every CTA gets the same estimated cost: a unit's
+// cost depends on its width (at r = 2 a unit holds four times the codes of
+// an r = 8 unit in the same bytes). A CTA walks its range one row block at a
+// time; a row block it owns whole is stored into y directly, a row block
+// shared with a neighbour is added into y with fp32 atomics, and the prep
+// kernel zeroes exactly those shared row blocks first.
 //
 // CTA = 8 consumer warps + 1 producer warp. The producer stages each unit in
 // shared memory with 1-D bulk copies (cp.async.bulk, one per row and plane)
@@ -21,7 +25,7 @@
 // exactly 2^e + c * 2^(e-7+p); choosing p and e so that the code weight is 1
 // (or 4, 16 for the high plane of r = 3, 6; 16 for the high nibble of r = 8)
 // gives the integer value off + weight*c, exact in bf16. The offsets "off"
-// sum to O_m = sum_k x[m,k] off(k), which depends only on k mod 8 and is
+// sum to O_m = sum_k x[m,k] off(k), which depends only on k mod 16 and is
 // removed in the epilogue from per-class activation sums computed once:
 //   y = A_n (acc - O_m) - B_n Sx_m,  A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n.
 // Offsets stay <= 384, so fp32 partial sums stay small (accuracy), and
@@ -52,6 +56,8 @@ constexpr int kMaxStages = 8;
 constexpr int kBarrierBytes = 256;  // barriers, abort flag; last 64 bytes: zero block
 constexpr int kMaxDynSmem = 227 * 1024;
 constexpr size_t kStageBudget = 110 * 1024;
+constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
+constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
 
 // Per-linear descriptor, passed by value in the kernel parameters.
 struct LinDesc {
@@ -61,7 +67,7 @@ struct LinDesc {
   const float* zero;
   float* y;
   const uint8_t* xf;   // activations in fragment order, n_kc blocks of M*KC bf16
-  const float* psum;   // [M][4] activation sums per class (k >> 1) & 3
+  const float* psum;   // [M][8] activation sums per class (k >> 1) & 7
   int N, K, r, kc, n_kc, unit_begin;
 };
 
@@ -76,6 +82,7 @@ struct GemvParams {
   int pitch0, pitch1;
   uint32_t* err;
   unsigned long long wait_ns;
+  int cta_begin[kMaxCtas + 1];  // unit range of CTA c: [cta_begin[c], cta_begin[c + 1])
   LinDesc lin[CAP];
 };
 
@@ -162,14 +169,18 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
   }
 }
 
-// Offset coefficients per activation class (k >> 1) & 3 for each width.
-__device__ __forceinline__ void offset_coeffs(int r, float (&c)[4]) {
-  switch (r) {
-    case 8: c[0] = c[1] = c[2] = c[3] = 384.f; break;
-    case 4: c[0] = c[1] = c[2] = c[3] = 16.f; break;
-    case 2: c[0] = 16.f; c[1] = 4.f; c[2] = 16.f; c[3] = 4.f; break;
-    case 3: c[0] = 80.f; c[1] = 36.f; c[2] = 32.f; c[3] = 12.f; break;
-    default: c[0] = 272.f; c[1] = 80.f; c[2] = 272.f; c[3] = 80.f; break;  // 6
+// Offset of the decoded value per activation class (k >> 1) & 7 for each
+// width (the sum over the planes of the magic added to the code). The codes
+// sit in the top mantissa bits, so the offsets stay small next to the code
+// unit (16 or 4 at r = 2): the fp32 sums then lose little to cancellation when
+// the offsets are taken out again.
+__device__ __forceinline__ void offset_coeffs(int r, float (&c)[kClasses]) {
+  constexpr float r2[4] = {16.f, 4.f, 16.f, 4.f};
+  constexpr float r3[4] = {80.f, 36.f, 32.f, 12.f};
+  constexpr float r6[4] = {272.f, 80.f, 272.f, 80.f};
+#pragma unroll
+  for (int i = 0; i < kClasses; ++i) {
+    c[i] = r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i & 3] : r == 3 ? r3[i & 3] : r6[i & 3];
   }
 }
 
@@ -291,13 +302,18 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
   }
 }
 
+// Epilogue of one row block of this warp's 16 rows: scales the raw sums,
+// removes the decoding offsets and the zero point (once per row, by the part
+// that starts at k-chunk 0) and writes y. A row block this CTA owns whole is
+// stored; a shared one is added atomically into y, which the prep kernel
+// zeroed.
 template <int NT, int CAP>
-__device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, int warp, int lane,
-                           float (&tot)[NT][4]) {
+__device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
+                           int lane, const float (&tot)[NT][4]) {
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
-  float c[4];
+  float c[kClasses];
   offset_coeffs(L.r, c);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -313,17 +329,64 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, int
         if (m >= p.M) continue;
         float v = tot[nt][2 * h + e];
         if (kc0 == 0) {
-          const float* P = L.psum + m * 4;
-          const float O = c[0] * P[0] + c[1] * P[1] + c[2] * P[2] + c[3] * P[3];
-          const float Sx = (P[0] + P[1]) + (P[2] + P[3]);
+          const float* P = L.psum + m * kClasses;
+          float O = 0.f, Sx = 0.f;
+#pragma unroll
+          for (int i = 0; i < kClasses; ++i) {
+            O = fmaf(c[i], P[i], O);
+            Sx += P[i];
+          }
           v = A * (v - O) - B * Sx;
         } else {
           v = A * v;
         }
-        atomicAdd(L.y + static_cast<int64_t>(m) * L.N + n, v);
+        float* dst = L.y + static_cast<int64_t>(m) * L.N + n;
+        if (whole) *dst = v;
+        else atomicAdd(dst, v);
       }
     }
   }
+}
+
+// Consumes `seg` consecutive staged units of one row block at width R and
+// adds them into `tot`. The two MMA accumulator chains are folded into `tot`
+// after every unit, which keeps each fp32 chain short. Returns false if a wait
+// gave up (the abort flag is then set for the whole CTA).
+template <int R, int NT, int NSUB, int CAP>
+__device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint8_t* stages,
+                                            uint64_t* full, uint64_t* empty,
+                                            volatile int* s_abort, int seg, int& s, uint32_t& ph,
+                                            bool active, const uint32_t (&xaddr)[NT],
+                                            const uint32_t (&xstep)[NT], int warp, int lane,
+                                            float (&tot)[NT][4]) {
+  for (int i = 0; i < seg; ++i) {
+    if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
+      if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
+      return false;
+    }
+    if (active) {
+      const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+      const uint32_t xs = smem_u32(st + p.off_x);
+      uint32_t xa[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) xa[nt] = xstep[nt] ? xs + xaddr[nt] : xaddr[nt];
+      float ch[NT][2][4];
+#pragma unroll
+      for (int b = 0; b < NT; ++b)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { ch[b][0][j] = 0.f; ch[b][1][j] = 0.f; }
+      process_unit<R, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane,
+                                ch);
+#pragma unroll
+      for (int b = 0; b < NT; ++b)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot[b][j] += ch[b][0][j] + ch[b][1][j];
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == p.stages) { s = 0; ph ^= 1u; }
+  }
+  return true;
 }
 
 template <int NT, int CAP>
@@ -349,9 +412,8 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(zero_block)[threadIdx.x] = 0u;
   __syncthreads();
 
-  const int64_t G = gridDim.x, cta = blockIdx.x;
-  const int u0 = static_cast<int>(int64_t(p.total_units) * cta / G);
-  const int u1 = static_cast<int>(int64_t(p.total_units) * (cta + 1) / G);
+  const int u0 = p.cta_begin[blockIdx.x];
+  const int u1 = p.cta_begin[blockIdx.x + 1];
   if (u0 >= u1) return;
 
   if (warp == kConsumerWarps) {
@@ -432,65 +494,44 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       xstep[nt] = static_cast<uint32_t>(p.M) * 64u;
     }
   }
-  float ch[NT][2][4];
-  float tot[NT][4];
-#pragma unroll
-  for (int b = 0; b < NT; ++b)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) { ch[b][0][i] = 0.f; ch[b][1][i] = 0.f; tot[b][i] = 0.f; }
-
+  // Sub-steps per unit: the low plane holds 192 bytes per row per unit for
+  // M <= 8 (3 sub-steps of 64 bytes) and 64 bytes for larger M.
+  constexpr int NSUB = (NT == 1) ? 3 : 1;
   Cursor c;
   cursor_init(p, u0, c);
-  int cur_l = c.l, cur_rb = c.rb, cur_kc0 = c.kc;
-  bool aborted = false;
-  int it = 0;
-  for (int u = u0; u < u1; ++u, ++it) {
-    const int s = it % S;
-    if (*s_abort || !mbar_wait_bounded(&full[s], (it / S) & 1, p.wait_ns)) {
-      if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
-      aborted = true;
-      break;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int u = u0; u < u1;) {
+    // One row block: units kc0 .. kc0 + seg - 1 of (linear c.l, row block c.rb).
+    const int seg = min(c.n_kc - c.kc, u1 - u);
+    const int kc0 = c.kc;
+    const bool whole = kc0 == 0 && seg == c.n_kc;
+    const bool active = warp * kRowsPerWarp < c.N - c.rb * kRowsPerUnit;
+    float tot[NT][4];
+#pragma unroll
+    for (int b = 0; b < NT; ++b)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tot[b][i] = 0.f;
+    bool ok;
+    switch (c.r) {
+      case 2: ok = run_segment<2, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 4: ok = run_segment<4, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 8: ok = run_segment<8, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 3: ok = run_segment<3, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      default: ok = run_segment<6, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
     }
-    if (c.l != cur_l || c.rb != cur_rb) {
-      flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
-#pragma unroll
-      for (int b = 0; b < NT; ++b)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tot[b][i] = 0.f;
-      cur_l = c.l; cur_rb = c.rb; cur_kc0 = c.kc;
-    }
-    const int rows = c.N - c.rb * kRowsPerUnit;
-    if (warp * kRowsPerWarp < rows) {
-      const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
-      const uint32_t xs = smem_u32(st + p.off_x);
-      uint32_t xa[NT];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) xa[nt] = xstep[nt] ? xs + xaddr[nt] : xaddr[nt];
-      // Sub-steps per unit: the low plane holds 192 bytes per row per unit
-      // for M <= 8 (3 sub-steps of 64 bytes) and 64 bytes for larger M.
-      constexpr int NSUB = (NT == 1) ? 3 : 1;
-      switch (c.r) {
-        case 2: process_unit<2, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
-        case 4: process_unit<4, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
-        case 8: process_unit<8, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
-        case 3: process_unit<3, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
-        default: process_unit<6, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane, ch); break;
+    if (!ok) break;  // outputs are undefined after a give-up; the flag says so
+    if (active) flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot);
+    u += seg;
+    c.kc += seg;
+    if (c.kc == c.n_kc) {
+      c.kc = 0;
+      if (++c.rb == c.nrb) {
+        c.rb = 0;
+        if (++c.l < p.n_lin) cursor_load(p, c);
       }
-      // Fold the two MMA chains into the row totals once per unit.
-#pragma unroll
-      for (int b = 0; b < NT; ++b)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          tot[b][i] += ch[b][0][i] + ch[b][1][i];
-          ch[b][0][i] = 0.f;
-          ch[b][1][i] = 0.f;
-        }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    cursor_next(p, c);
   }
-  if (!aborted) flush_rows<NT>(p, cur_l, cur_rb, cur_kc0, warp, lane, tot);
 }
 
 // ------------------------------------------------------------------ prep
@@ -505,20 +546,23 @@ struct PrepSum {
   float* psum;
   int K;
 };
+// A row block of an output that two or more CTAs add into: y[m, 128 rb ..
+// 128 rb + 127] for every m (columns past N excluded).
 struct PrepZero {
   float* y;
-  int64_t count;
+  int N, rb;
 };
 template <int CAP>
 struct PrepParams {
   int M, n_layout, n_sum, n_zero;
   PrepLayout lay[CAP];
   PrepSum sum[CAP];
-  PrepZero zero[CAP];
+  PrepZero zero[kMaxCtas];
 };
 
 // Builds the fragment-ordered activation blocks (zero-padded to whole
-// k-chunks), the per-class activation sums and zeroes every output.
+// k-chunks) and the per-class activation sums, and zeroes the output row
+// blocks that several CTAs add into.
 template <int CAP>
 __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ PrepParams<CAP> p) {
   pdl_launch_dependents();
@@ -529,7 +573,9 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
     const int m = blockIdx.x % M;
     const __nv_bfloat16* row = J.x + int64_t(m) * J.K;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    // 8 consecutive elements k0..k0+7 (k0 % 8 == 0): classes 0,0,1,1,2,2,3,3
+    // 8 consecutive elements k0..k0+7 (k0 % 8 == 0) fall in classes
+    // 4h, 4h, 4h+1, 4h+1, ..., 4h+3 with h = (k0 >> 3) & 1; the stride of
+    // the loop is a multiple of 16, so h is the parity of the thread.
     for (int k0 = threadIdx.x * 8; k0 < J.K; k0 += blockDim.x * 8) {
       const uint4 u = *reinterpret_cast<const uint4*>(row + k0);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -537,19 +583,20 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       for (int i = 0; i < 4; ++i)
         acc[i] += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
     }
-    __shared__ float red[4][8];
+    __shared__ float red[kClasses][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float v = acc[i];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if ((threadIdx.x & 31) == 0) red[i][threadIdx.x >> 5] = v;
+      for (int o = 16; o > 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);  // same parity
+      const int lane = threadIdx.x & 31;
+      if (lane < 2) red[4 * lane + i][threadIdx.x >> 5] = v;
     }
     __syncthreads();
-    if (threadIdx.x < 4) {
+    if (threadIdx.x < kClasses) {
       float v = 0.f;
       for (int w8 = 0; w8 < (int)(blockDim.x >> 5); ++w8) v += red[threadIdx.x][w8];
-      J.psum[m * 4 + threadIdx.x] = v;
+      J.psum[m * kClasses + threadIdx.x] = v;
     }
   }
   // (2) fragment-ordered activation groups: thread per (layout, m, 8-code group)
@@ -580,11 +627,14 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       *reinterpret_cast<uint4*>(L.xf + off) = v;
     }
   }
-  // (3) zero the outputs
-  for (int zi = 0; zi < p.n_zero; ++zi) {
-    float* y = p.zero[zi].y;
-    const int64_t cnt = p.zero[zi].count;
-    for (int64_t i = tid; i < cnt; i += stride) y[i] = 0.f;
+  // (3) zero the shared output row blocks
+  const int64_t zt = int64_t(p.n_zero) * M * kRowsPerUnit;
+  for (int64_t i = tid; i < zt; i += stride) {
+    const PrepZero& Z = p.zero[i / (int64_t(M) * kRowsPerUnit)];
+    const int rem = static_cast<int>(i % (int64_t(M) * kRowsPerUnit));
+    const int m = rem / kRowsPerUnit;
+    const int n = Z.rb * kRowsPerUnit + rem % kRowsPerUnit;
+    if (n < Z.N) Z.y[int64_t(m) * Z.N + n] = 0.f;
   }
 }
 
@@ -597,9 +647,10 @@ struct KernelCache {
 };
 std::mutex g_cache_mutex;
 
+// Persistent grid for `units` work units at `smem` bytes of shared memory:
+// every resident CTA slot of the device, at most one CTA per unit.
 template <int NT, int CAP>
-cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int sms, int units,
-                        cudaStream_t stream) {
+cudaError_t gemv_grid(size_t smem, int sms, int units, int* grid_out) {
   auto kern = gemv_streamk_kernel<NT, CAP>;
   static std::map<int, KernelCache> caches;
   int dev = 0;
@@ -624,7 +675,13 @@ cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int sms, int uni
     }
     occ = it->second;
   }
-  const int grid = std::max(1, std::min(units, sms * occ));
+  *grid_out = std::max(1, std::min(std::min(units, sms * occ), kMaxCtas));
+  return cudaSuccess;
+}
+
+template <int NT, int CAP>
+cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int grid, cudaStream_t stream) {
+  auto kern = gemv_streamk_kernel<NT, CAP>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -688,6 +745,21 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
   g_map_tables.emplace(std::move(k2), dptr);
   *out = dptr;
   return cudaSuccess;
+}
+
+// Relative cost of one unit of each width, for cutting the CTA ranges. A unit
+// always holds the same plane bytes per row (two planes hold 1.5x), while the
+// decode and MMA work grows with the codes in it: measured per-unit times of
+// single-width stacks on B200 at M = 1 put r = 2 at about 1.6x and r = 4 at
+// about 1.1x an r = 8 unit; r = 3 and 6 are estimated from their planes.
+int64_t unit_cost(int r) {
+  switch (r) {
+    case 8: return 100;
+    case 4: return 108;
+    case 2: return 157;
+    case 6: return 170;
+    default: return 280;  // 3
+  }
 }
 
 template <int CAP>
@@ -758,7 +830,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     if (em != cudaSuccess) return em;
   }
   const size_t psum_off = xf_bytes;
-  const size_t ws_bytes = psum_off + size_t(n_sums) * M * 4 * sizeof(float) + 256;
+  const size_t ws_bytes = psum_off + size_t(n_sums) * M * kClasses * sizeof(float) + 256;
   void* ws = nullptr;
   cudaError_t e = cudaSuccess;
   if (fixed) {
@@ -772,29 +844,8 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   float* psum_base = reinterpret_cast<float*>(wsb + psum_off);
   for (int i = 0; i < n_jobs; ++i) {
     gp.lin[i].xf = wsb + layouts[lay_of[i]].off;
-    gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * 4;
+    gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * kClasses;
   }
-
-  // Prep launch.
-  pp.M = M;
-  pp.n_layout = n_layouts;
-  pp.n_sum = n_sums;
-  pp.n_zero = n_jobs;
-  for (int i = 0; i < n_layouts; ++i) {
-    pp.lay[i] = {static_cast<const __nv_bfloat16*>(layouts[i].x), wsb + layouts[i].off,
-                 layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc,
-                 layouts[i].b0 == 8 ? 1 : 0};
-  }
-  for (int i = 0; i < n_sums; ++i) {
-    pp.sum[i] = {static_cast<const __nv_bfloat16*>(sum_x[i]), psum_base + size_t(i) * M * 4, sum_k[i]};
-  }
-  for (int i = 0; i < n_jobs; ++i) pp.zero[i] = {jobs[i].y, int64_t(M) * jobs[i].N};
-  const int sms = sm_count();
-  int prep_grid = std::max(n_sums * M, sms);
-  prep_grid = std::min(prep_grid, 4 * sms);
-  gemv_prep_kernel<CAP><<<prep_grid, 256, 0, stream>>>(pp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
 
   // Stage layout: [128 rows x P0][128 rows x P1][M x KC bf16 activations].
   const int P1 = two_planes ? P0 / 2 : 0;
@@ -806,6 +857,77 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   int stages = static_cast<int>(kStageBudget / stage_bytes);
   stages = std::max(2, std::min(stages, kMaxStages));
   const size_t smem = kBarrierBytes + size_t(stages) * stage_bytes;
+  const int sms = sm_count();
+  int grid = 1;
+  switch (NT) {
+    case 1: e = gemv_grid<1, CAP>(smem, sms, units, &grid); break;
+    case 2: e = gemv_grid<2, CAP>(smem, sms, units, &grid); break;
+    case 3: e = gemv_grid<3, CAP>(smem, sms, units, &grid); break;
+    default: e = gemv_grid<4, CAP>(smem, sms, units, &grid); break;
+  }
+  if (e != cudaSuccess) return e;
+
+  // CTA ranges of equal estimated cost, and the row blocks they share.
+  int64_t total_cost = 0;
+  for (int i = 0; i < n_jobs; ++i) {
+    const int64_t lin_units = (i + 1 < n_jobs ? gp.lin[i + 1].unit_begin : units) - gp.lin[i].unit_begin;
+    total_cost += lin_units * unit_cost(jobs[i].r);
+  }
+  int n_zero = 0;
+  {
+    int li = 0;
+    int64_t cost_before = 0;  // cost of the units before linear li
+    for (int c = 0; c <= grid; ++c) {
+      const int64_t target = (total_cost * c + grid - 1) / grid;  // ceil(c T / G)
+      // first unit whose preceding cost reaches the target
+      while (li < n_jobs) {
+        const int64_t lin_units = (li + 1 < n_jobs ? gp.lin[li + 1].unit_begin : units) - gp.lin[li].unit_begin;
+        const int64_t lin_cost = lin_units * unit_cost(jobs[li].r);
+        if (target <= cost_before + lin_cost) break;
+        cost_before += lin_cost;
+        ++li;
+      }
+      int u;
+      if (li >= n_jobs) {
+        u = units;
+      } else {
+        const int64_t w = unit_cost(jobs[li].r);
+        u = gp.lin[li].unit_begin + static_cast<int>((target - cost_before + w - 1) / w);
+      }
+      if (c == 0) u = 0;
+      if (c == grid) u = units;
+      gp.cta_begin[c] = u;
+      if (c > 0 && c < grid && u < units && li < n_jobs) {
+        const LinDesc& L = gp.lin[li];
+        const int local = u - L.unit_begin;
+        if (local % L.n_kc != 0) {
+          const int rb = local / L.n_kc;
+          if (n_zero == 0 || pp.zero[n_zero - 1].y != L.y || pp.zero[n_zero - 1].rb != rb)
+            pp.zero[n_zero++] = {L.y, L.N, rb};
+        }
+      }
+    }
+  }
+
+  // Prep launch.
+  pp.M = M;
+  pp.n_layout = n_layouts;
+  pp.n_sum = n_sums;
+  pp.n_zero = n_zero;
+  for (int i = 0; i < n_layouts; ++i) {
+    pp.lay[i] = {static_cast<const __nv_bfloat16*>(layouts[i].x), wsb + layouts[i].off,
+                 layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc,
+                 layouts[i].b0 == 8 ? 1 : 0};
+  }
+  for (int i = 0; i < n_sums; ++i) {
+    pp.sum[i] = {static_cast<const __nv_bfloat16*>(sum_x[i]),
+                 psum_base + size_t(i) * M * kClasses, sum_k[i]};
+  }
+  int prep_grid = std::max(n_sums * M, sms);
+  prep_grid = std::min(prep_grid, 4 * sms);
+  gemv_prep_kernel<CAP><<<prep_grid, 256, 0, stream>>>(pp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
 
   gp.n_lin = n_jobs;
   gp.M = M;
@@ -827,10 +949,10 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.wait_ns = wait_limit_ns();
 
   switch (NT) {
-    case 1: return launch_gemv<1, CAP>(gp, smem, sms, units, stream);
-    case 2: return launch_gemv<2, CAP>(gp, smem, sms, units, stream);
-    case 3: return launch_gemv<3, CAP>(gp, smem, sms, units, stream);
-    default: return launch_gemv<4, CAP>(gp, smem, sms, units, stream);
+    case 1: return launch_gemv<1, CAP>(gp, smem, grid, stream);
+    case 2: return launch_gemv<2, CAP>(gp, smem, grid, stream);
+    case 3: return launch_gemv<3, CAP>(gp, smem, grid, stream);
+    default: return launch_gemv<4, CAP>(gp, smem, grid, stream);
   }
 }
 
@@ -852,7 +974,7 @@ size_t gemv_scratch_bytes(const LinearJob& job, int M) {
   const int64_t n_kc = (job.K + kc - 1) / kc;
   size_t xf = size_t(n_kc) * M * kc * 2;
   xf = (xf + 255) & ~size_t(255);
-  return xf + size_t(M) * 4 * sizeof(float) + 256;
+  return xf + size_t(M) * kClasses * sizeof(float) + 256;
 }
 
 cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
