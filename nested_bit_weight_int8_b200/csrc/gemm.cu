@@ -1,13 +1,432 @@
-// Prefill path (M > 32). The tcgen05 GEMM lands here.
+// Prefill path (M > 32): y = x . W_r^T with W_r[n,k] = alpha_n (S(q[n,k], r) - z_n)
+// on the fifth-generation tensor cores ("Matryoshka Quantization" explainer
+// page: Eq. 1 dequantization alpha*(q - z), Eq. 6 slicing; "Mix'n'Match and
+// Interpolative Slicing" for the widths 6 and 3 served from the same int8
+// container).
+//
+// With codes c[n,k] = S(q[n,k], r) / 2^(8-r), the product factors as
+//   y[m,n] = A_n * sum_k x[m,k] c[n,k] - B_n * Sx[m],
+//   A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n,  Sx[m] = sum_k x[m,k],
+// so the contraction runs on exact integer operands: every code is an
+// integer below 256, exact in bf16, and products and sums are fp32.
+//
+// Tile: 128 weight rows (n) x 128 batch rows (m), K in stages of 128 codes.
+// The weights are the MMA's A operand and live in tensor memory; x is the B
+// operand in shared memory (128-byte swizzled, K-major), so D = W x^T sits in
+// tensor memory with one weight row per lane and one batch row per column.
+//   warp 0      : TMA producer (x box, plane boxes) into a ring of stages
+//   warp 1      : allocates tensor memory, issues tcgen05.mma (one thread)
+//   warps 4..11 : decode: each thread owns one weight row (its TMEM lane) and
+//                 half of the stage's codes, unpacks them from the staged
+//                 planes to bf16 and writes them to tensor memory
+//                 (tcgen05.st); then the same warps run the epilogue.
+// Every mbarrier wait is bounded; a wait that gives up sets the device error
+// word, the CTA drains its copies and MMAs, frees its tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cstdint>
+#include <map>
+#include <mutex>
+
+#include "mq_device.cuh"
 #include "mq_internal.h"
+#include "tc05.cuh"
 
 namespace mq {
+namespace {
+
+constexpr int kBN = 128;          // weight rows per CTA (MMA M, TMEM lanes)
+constexpr int kBM = 128;          // batch rows per CTA (MMA N, TMEM columns)
+constexpr int kBK = 128;          // codes of K per stage
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 12 * 32;
+constexpr int kDecodeWarp0 = 4;   // warps 4..11 decode, then run the epilogue
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;                 // D: columns [0, 128)
+constexpr uint32_t kASlotCol = 128;             // A slot s: columns [128 + 64 s, +64)
+constexpr uint32_t kXStageBytes = kBM * kBK * 2;      // two 64-code swizzled sub-tiles
+constexpr uint32_t kXSubBytes = kBM * 64 * 2;         // 16 KB
+constexpr uint32_t kHeaderBytes = 1024;
+
+struct GemmParams {
+  CUtensorMap map_x;       // x: M x K bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap map_p0;      // plane 0: N rows x K*b0/8 bytes, box 16*b0 x 128
+  CUtensorMap map_p1;      // plane 1 (widths 3, 6)
+  const float* alpha;
+  const float* zero;
+  const float* sx;         // Sx[m] = sum_k x[m,k]
+  float* y;                // M x N fp32
+  uint32_t* err;
+  unsigned long long wait_ns;
+  int M, N, K, r;
+  uint32_t stage_bytes;    // x sub-tiles + plane 0 box + plane 1 box, 1024-aligned
+  uint32_t off_p0, off_p1; // plane boxes within a stage
+};
+
+// ------------------------------------------------------------ Sx kernel
+// Sx[m] = sum_k x[m,k] in fp32, one CTA per batch row.
+__global__ void __launch_bounds__(256) rowsum_kernel(const __nv_bfloat16* __restrict__ x, int K,
+                                                     float* __restrict__ sx) {
+  const __nv_bfloat16* row = x + static_cast<int64_t>(blockIdx.x) * K;
+  float acc = 0.f;
+  for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + k0);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      acc += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) v += red[i];
+    sx[blockIdx.x] = v;
+  }
+}
+
+// ------------------------------------------------------------ decode
+// bf16x2 128.0 in both halves: OR-ing a code c < 128 into the mantissa gives
+// 128 + c exactly; subtracting 128 again leaves the integer c.
+constexpr uint32_t kMag128x2 = 0x43004300u;
+
+__device__ __forceinline__ uint32_t exact_pair(uint32_t codes2) {
+  uint32_t d;
+  // bf16x2 subtract (exact: both operands and the result are small integers)
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(codes2 | kMag128x2), "r"(kMag128x2));
+  return d;
+}
+
+// Two container bytes (0..255) as an exact bf16x2 pair, through fp32:
+// 2^23 + c is built by placing c in the low mantissa byte.
+__device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
+  const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - 8388608.0f;
+  const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - 8388608.0f;
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// Unpacks 64 consecutive codes of one weight row into 32 bf16x2 registers
+// (register j holds codes 2j, 2j+1: the even code in the low half, as the
+// A operand in tensor memory expects). `p0` / `p1` point at this row's 64-code
+// slice of plane 0 / plane 1 in shared memory. Plane word layout: local code
+// u of a width-b word sits at bit 16*(u%2) + b*(u/2) (b < 8), at 8u for b = 8.
+template <int R>
+__device__ __forceinline__ void decode64(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[32]) {
+  if constexpr (R == 2) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u);
+  } else if constexpr (R == 4) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu);
+  } else if constexpr (R == 3) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint2 h = *reinterpret_cast<const uint2*>(p1);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t u[2] = {h.x, h.y};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t lo = (w[j / 8] >> (2 * (j % 8))) & 0x00030003u;
+      const uint32_t hi = ((u[j / 16] >> (j % 16)) & 0x00010001u) << 2;
+      v[j] = exact_pair(lo | hi);
+    }
+  } else if constexpr (R == 6) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint4 h = *reinterpret_cast<const uint4*>(p1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t u[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t lo = (w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu;
+      const uint32_t hi = ((u[j / 8] >> (2 * (j % 8))) & 0x00030003u) << 4;
+      v[j] = exact_pair(lo | hi);
+    }
+  } else {  // R == 8: bytes, 4 codes per word
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 a = *reinterpret_cast<const uint4*>(p0 + 16 * i);
+      w[4 * i] = a.x; w[4 * i + 1] = a.y; w[4 * i + 2] = a.z; w[4 * i + 3] = a.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = (j % 2 == 0) ? exact_pair_bytes(w[j / 2], 0x7440u, 0x7441u)
+                          : exact_pair_bytes(w[j / 2], 0x7442u, 0x7443u);
+  }
+}
+
+
+// ------------------------------------------------------------ kernel
+template <int R>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base: the swizzled x sub-tiles need it.
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // TMA -> decode
+  uint64_t* decoded = full + kStages;                        // decode -> MMA
+  uint64_t* empty = decoded + kStages;                       // MMA -> TMA, decode
+  uint64_t* acc_full = empty + kStages;                      // MMA -> epilogue
+  uint64_t* drain = acc_full + 1;                            // MMA completion at exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* stages = smem + kHeaderBytes;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+  const int n_k = p.K / kBK;
+  constexpr int kDecodeWarps = 8;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&decoded[i], kDecodeWarps);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc05::alloc(smem_u32(tmem_slot), kTmemCols);
+    tc05::relinquish();
+    tc05::fence_before_sync();
+  }
+  __syncthreads();
+  tc05::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&p.map_x);
+      prefetch_tmap(&p.map_p0);
+      int issued = 0;
+      const uint32_t p0_bytes = 128u * 16u * (R == 8 ? 8 : (R == 4 || R == 6) ? 4 : 2);
+      const uint32_t p1_bytes = (R == 3) ? 128u * 16u : (R == 6) ? 128u * 32u : 0u;
+      for (int it = 0; it < n_k; ++it, ++issued) {
+        const int s = it % kStages;
+        if (it >= kStages &&
+            (*s_abort || !mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, p.wait_ns))) {
+          atomicOr(p.err, kErrWaitEmpty);
+          *s_abort = 1;
+          break;
+        }
+        uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], kXStageBytes + p0_bytes + p1_bytes);
+        const int k0 = it * kBK;
+        tma_load_2d(st, &p.map_x, k0, m0, &full[s]);
+        tma_load_2d(st + kXSubBytes, &p.map_x, k0 + 64, m0, &full[s]);
+        tma_load_2d(st + p.off_p0, &p.map_p0, it * static_cast<int>(p0_bytes / 128u), n0, &full[s]);
+        if (p1_bytes) tma_load_2d(st + p.off_p1, &p.map_p1, it * static_cast<int>(p1_bytes / 128u), n0, &full[s]);
+      }
+      // no bulk copy may be in flight when this thread leaves
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int j = first; j < issued; ++j)
+        if (!mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc05::idesc_bf16_f32(kBN, kBM);
+      bool ok = true;
+      for (int it = 0; it < n_k; ++it) {
+        const int s = it % kStages;
+        if (*s_abort || !mbar_wait_bounded(&decoded[s], (it / kStages) & 1, p.wait_ns)) {
+          atomicOr(p.err, kErrMma);
+          *s_abort = 1;
+          ok = false;
+          break;
+        }
+        tc05::fence_after_sync();
+        const uint32_t xs = smem_u32(stages + static_cast<size_t>(s) * p.stage_bytes);
+#pragma unroll
+        for (int j = 0; j < kBK / 16; ++j) {
+          // k16 step j: A columns advance by 8 (two bf16 per column); B stays in
+          // sub-tile j / 4 and advances 32 bytes along its 128-byte rows.
+          const uint64_t bdesc = tc05::desc_kmajor_sw128(xs + (j / 4) * kXSubBytes + (j % 4) * 32);
+          tc05::mma_ts(tmem + kAccCol, tmem + kASlotCol + s * 64 + j * 8, bdesc, idesc,
+                       it > 0 || j > 0);
+        }
+        tc05::commit(smem_u32(&empty[s]));
+      }
+      if (ok) tc05::commit(smem_u32(acc_full));
+      // all MMAs this thread issued have finished before the CTA moves on
+      tc05::commit(smem_u32(drain));
+      if (!mbar_wait_bounded(drain, 0, 1000000000ull)) atomicOr(p.err, kErrDrain);
+    }
+  } else if (warp >= kDecodeWarp0) {
+    // ---------------------------------------------------------- decode
+    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    const int h = (warp - kDecodeWarp0) >> 2;  // which 64 codes of the stage
+    const int row = 32 * q + lane;             // weight row within the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    constexpr int b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
+    constexpr int b1 = (R == 3) ? 1 : (R == 6) ? 2 : 0;
+    bool ok = true;
+    for (int it = 0; it < n_k; ++it) {
+      const int s = it % kStages;
+      // Every lane waits (each needs the barrier's ordering for the staged
+      // bytes); the warp then decides together, since the tensor-memory
+      // store below must be executed by all of its lanes.
+      bool mine = *s_abort == 0 && mbar_wait_bounded(&full[s], (it / kStages) & 1, p.wait_ns) &&
+                  (it < kStages || mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, p.wait_ns));
+      if (!__all_sync(0xffffffffu, mine)) {
+        if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
+        ok = false;
+        break;
+      }
+      const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+      const uint8_t* r0 = st + p.off_p0 + row * (16 * b0) + h * (8 * b0);
+      const uint8_t* r1 = st + p.off_p1 + row * (16 * (b1 ? b1 : 1)) + h * (8 * (b1 ? b1 : 1));
+      uint32_t v[32];
+      decode64<R>(r0, r1, v);
+      tc05::st_32x32b_x32(tmem + lane_addr + kASlotCol + s * 64 + h * 32, v);
+      tc05::wait_st();
+      tc05::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&decoded[s]);
+    }
+    // ---------------------------------------------------------- epilogue
+    // Warp (q, h) writes batch columns [64 h, 64 h + 64) of its 32 weight rows.
+    const bool acc_ready = ok && __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0, p.wait_ns));
+    if (acc_ready) {
+      tc05::fence_after_sync();
+      const int n = n0 + row;
+      const bool row_ok = n < p.N;
+      float A = 0.f, B = 0.f;
+      if (row_ok) {
+        const float a = __ldg(p.alpha + n);
+        A = a * static_cast<float>(1 << (8 - R));
+        B = a * __ldg(p.zero + n);
+      }
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const int col = 64 * h + 32 * c;
+        uint32_t d[32];
+        tc05::ld_32x32b_x32(tmem + lane_addr + kAccCol + col, d);
+        tc05::wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m0 + col + j;
+            if (m < p.M) {
+              const float sx = __ldg(p.sx + m);
+              p.y[static_cast<int64_t>(m) * p.N + n] = A * __uint_as_float(d[j]) - B * sx;
+            }
+          }
+        }
+      }
+    } else if (ok) {
+      if (lane == 0) { atomicOr(p.err, kErrMma); *s_abort = 1; }
+    }
+    tc05::fence_before_sync();
+  }
+  if (warp == 1) tc05::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc05::fence_after_sync();
+    tc05::dealloc(tmem, kTmemCols);
+  }
+}
+
+
+template <int R>
+cudaError_t launch_gemm_r(const GemmParams& gp, dim3 grid, size_t smem, cudaStream_t stream) {
+  auto kern = gemm_tc05_kernel<R>;
+  static std::mutex mu;
+  static std::map<int, bool> attr_set;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  kern<<<grid, kGemmThreads, smem, stream>>>(gp);
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
-  (void)job; (void)M; (void)stream;
-  return cudaErrorNotSupported;
+  if (M < 1 || job.K % kBK != 0 || job.N < 1) return cudaErrorNotSupported;
+  if ((job.N + kBN - 1) / kBN > 0x7FFFFFFF || (M + kBM - 1) / kBM > 65535) return cudaErrorNotSupported;
+  int b0, b1;
+  plane_widths(job.r, b0, b1);
+  if (b0 == 0) return cudaErrorInvalidValue;
+
+  static thread_local GemmParams gp;
+  cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, true);
+  if (e != cudaSuccess) return e;
+  e = encode_map_2d(&gp.map_p0, job.packed, uint64_t(job.N), uint64_t(job.K) * b0 / 8,
+                    16u * b0, kBN, 1);
+  if (e != cudaSuccess) return e;
+  if (b1) {
+    e = encode_map_2d(&gp.map_p1, job.packed + job.N * job.K * b0 / 8, uint64_t(job.N),
+                      uint64_t(job.K) * b1 / 8, 16u * b1, kBN, 1);
+    if (e != cudaSuccess) return e;
+  } else {
+    gp.map_p1 = gp.map_p0;
+  }
+
+  void* ws = nullptr;
+  e = get_workspace(stream, size_t(M) * sizeof(float) + 256, &ws);
+  if (e != cudaSuccess) return e;
+  float* sx = static_cast<float*>(ws);
+  uint32_t* err = nullptr;
+  e = get_error_word(&err);
+  if (e != cudaSuccess) return e;
+
+  gp.alpha = job.alpha;
+  gp.zero = job.zero;
+  gp.sx = sx;
+  gp.y = job.y;
+  gp.err = err;
+  gp.wait_ns = wait_limit_ns();
+  gp.M = M;
+  gp.N = static_cast<int>(job.N);
+  gp.K = static_cast<int>(job.K);
+  gp.r = job.r;
+  gp.off_p0 = kXStageBytes;
+  const uint32_t p0_bytes = 128u * 16u * b0;
+  gp.off_p1 = gp.off_p0 + p0_bytes;
+  const uint32_t p1_bytes = 128u * 16u * b1;
+  gp.stage_bytes = (gp.off_p1 + p1_bytes + 1023u) & ~1023u;
+  const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(kStages) * gp.stage_bytes;
+
+  rowsum_kernel<<<M, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(job.x),
+                                        static_cast<int>(job.K), sx);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const dim3 grid(static_cast<unsigned>((job.N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
+  switch (job.r) {
+    case 8: return launch_gemm_r<8>(gp, grid, smem, stream);
+    case 6: return launch_gemm_r<6>(gp, grid, smem, stream);
+    case 4: return launch_gemm_r<4>(gp, grid, smem, stream);
+    case 3: return launch_gemm_r<3>(gp, grid, smem, stream);
+    case 2: return launch_gemm_r<2>(gp, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace mq

@@ -48,10 +48,13 @@ uint64_t wait_limit_ns();
 void set_last_error(const char* msg);
 
 // 2-D tensor map over a row-major matrix of `rows` x `row_elems` elements of
-// `elem_bytes` bytes (1: uint8, 2: bf16), box `box_inner` x `box_rows`, no
-// swizzle, out-of-bounds elements read as zero. Cached per arguments.
+// `elem_bytes` bytes (1: uint8, 2: bf16), box `box_inner` x `box_rows`,
+// out-of-bounds elements read as zero, no swizzle unless `swizzle128` (then
+// the box rows are stored in 128-byte swizzled atoms; box_inner * elem_bytes
+// must be 128). Cached per arguments.
 cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t row_elems,
-                          uint32_t box_inner, uint32_t box_rows, int elem_bytes);
+                          uint32_t box_inner, uint32_t box_rows, int elem_bytes,
+                          bool swizzle128 = false);
 int sm_count();
 
 cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
@@ -79,7 +82,8 @@ size_t gemv_scratch_bytes(const LinearJob& job, int M);
 cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
                            const FixedScratch& scratch);
 
-// Prefill path (M > 32): tcgen05 GEMM for one linear.
+// Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
+// cudaErrorNotSupported for shapes it does not serve (nothing launched).
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);
 
 }  // namespace mq
