@@ -259,6 +259,9 @@ def rows_timings(dev, stream):
         tot = 0.0
         for _ in range(reps):
             flush.zero_()
+            # keep the GPU busy while the host enqueues the call, so that the
+            # events bracket device time only, not the host's launch latency
+            torch.cuda._sleep(200000)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -279,16 +282,29 @@ def rows_timings(dev, stream):
         out[f"slice_pack_r{r}"] = {"us": round(us, 2), "GBps": round((n * k + n * k * r // 8) / us / 1e3, 1)}
         us = timed(lambda: mq.linear(x, 1, k, p, a, z, n, r, y, stream))
         out[f"decode_linear_r{r}_M1"] = {"us": round(us, 2), "GBps": round(n * k * r / 8 / us / 1e3, 1)}
-    try:
-        m = 2048
-        xm = torch.randn((m, k), generator=gen, device=dev).to(torch.bfloat16)
-        ym = torch.empty((m, n), dtype=torch.float32, device=dev)
-        p = torch.empty(mq.packed_bytes(n, k, 4), dtype=torch.uint8, device=dev)
-        mq.slice_pack(q, n, k, 4, p, stream)
-        us = timed(lambda: mq.linear(xm, m, k, p, a, z, n, 4, ym, stream), reps=5)
-        out["prefill_gemm_r4_M2048"] = {"us": round(us, 2), "TFLOPs": round(2 * m * n * k / us / 1e6, 1)}
-    except mq.MQError as e:
-        out["prefill_gemm_r4_M2048"] = {"unavailable": str(e)}
+    # prefill GEMM on the 9B-shaped matrices, M = 2048, the interpolative widths
+    bf16_peak = _peaks()[1]
+    m = 2048
+    for name, n_p, k_p, seed in (("up", 14336, 3584, 500), ("down", 3584, 14336, 501)):
+        gen.manual_seed(seed)
+        w_p = (torch.randn((n_p, k_p), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        q_p = torch.empty((n_p, k_p), dtype=torch.uint8, device=dev)
+        a_p = torch.empty(n_p, dtype=torch.float32, device=dev)
+        z_p = torch.empty(n_p, dtype=torch.float32, device=dev)
+        mq.quantize_int8(w_p, mq.MQ_BF16, n_p, k_p, q_p, a_p, z_p, stream)
+        del w_p
+        xm = torch.randn((m, k_p), generator=gen, device=dev).to(torch.bfloat16)
+        ym = torch.empty((m, n_p), dtype=torch.float32, device=dev)
+        for r in (6, 4, 3, 2):
+            p_p = torch.empty(mq.packed_bytes(n_p, k_p, r), dtype=torch.uint8, device=dev)
+            mq.slice_pack(q_p, n_p, k_p, r, p_p, stream)
+            us = timed(lambda: mq.linear(xm, m, k_p, p_p, a_p, z_p, n_p, r, ym, stream), reps=5)
+            tf = 2 * m * n_p * k_p / us / 1e6
+            out[f"prefill_{name}_{n_p}x{k_p}_r{r}_M{m}"] = {
+                "us": round(us, 2), "TFLOPs": round(tf, 1),
+                "frac_of_bf16_peak": round(tf / bf16_peak, 3)}
+            del p_p
+        del q_p, xm, ym
     torch.cuda.synchronize()
     return out
 
@@ -510,6 +526,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--rows-only", action="store_true",
+                    help="time only the separate rows (quantize, slice-pack, one decode linear, "
+                         "prefill GEMMs) and print them; small enough for profiler captures")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -518,6 +537,15 @@ def main(argv=None):
         world = int(os.environ.get("WORLD_SIZE", "1"))
         if int(os.environ.get("RANK", "0")) == 0:
             print(json.dumps(run_reference(args, 0, world)), flush=True)
+        return 0
+    if args.rows_only:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        stream = torch.cuda.Stream(device=dev)
+        with torch.cuda.stream(stream):
+            rows = rows_timings(dev, stream)
+        print(json.dumps({"rows": rows}), flush=True)
         return 0
     rank, world, local = dist_setup(args.gpus)
     try:
