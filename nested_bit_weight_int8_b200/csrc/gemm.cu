@@ -10,14 +10,17 @@
 // so the contraction runs on exact integer operands: every code is an
 // integer below 256, exact in bf16, and products and sums are fp32.
 //
-// Tile: 128 weight rows (n) x 128 batch rows (m), K in stages of 128 codes.
+// Tile: 128 weight rows (n) x 256 batch rows (m), K in stages of 64 codes.
 // The weights are the MMA's A operand and live in tensor memory; x is the B
 // operand in shared memory (128-byte swizzled, K-major), so D = W x^T sits in
 // tensor memory with one weight row per lane and one batch row per column.
+// The 256-wide batch tile (the largest MMA N) spends each decoded weight on
+// twice the arithmetic of a square tile: the decode is ALU work that must
+// stay below the MMA time of a stage.
 //   warp 0      : TMA producer (x box, plane boxes) into a ring of stages
 //   warp 1      : allocates tensor memory, issues tcgen05.mma (one thread)
 //   warps 4..11 : decode: each thread owns one weight row (its TMEM lane) and
-//                 half of the stage's codes, unpacks them from the staged
+//                 32 of the stage's 64 codes, unpacks them from the staged
 //                 planes to bf16 and writes them to tensor memory
 //                 (tcgen05.st); then the same warps run the epilogue.
 // Every mbarrier wait is bounded; a wait that gives up sets the device error
@@ -39,22 +42,21 @@ namespace mq {
 namespace {
 
 constexpr int kBN = 128;          // weight rows per CTA (MMA M, TMEM lanes)
-constexpr int kBM = 128;          // batch rows per CTA (MMA N, TMEM columns)
-constexpr int kBK = 128;          // codes of K per stage
-constexpr int kStages = 4;
+constexpr int kBM = 256;          // batch rows per CTA (MMA N, TMEM columns)
+constexpr int kBK = 64;           // codes of K per stage
+constexpr int kStages = 5;
 constexpr int kGemmThreads = 12 * 32;
 constexpr int kDecodeWarp0 = 4;   // warps 4..11 decode, then run the epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;                 // D: columns [0, 128)
-constexpr uint32_t kASlotCol = 128;             // A slot s: columns [128 + 64 s, +64)
-constexpr uint32_t kXStageBytes = kBM * kBK * 2;      // two 64-code swizzled sub-tiles
-constexpr uint32_t kXSubBytes = kBM * 64 * 2;         // 16 KB
+constexpr uint32_t kAccCol = 0;                 // D: columns [0, 256)
+constexpr uint32_t kASlotCol = 256;             // A slot s: columns [256 + 32 s, +32)
+constexpr uint32_t kXStageBytes = kBM * kBK * 2;      // one 64-code swizzled tile, 32 KB
 constexpr uint32_t kHeaderBytes = 1024;
 
 struct GemmParams {
-  CUtensorMap map_x;       // x: M x K bf16, box 64 x 128, 128-byte swizzle
-  CUtensorMap map_p0;      // plane 0: N rows x K*b0/8 bytes, box 16*b0 x 128
-  CUtensorMap map_p1;      // plane 1 (widths 3, 6)
+  CUtensorMap map_x;       // x: M x K bf16, box 64 x 256, 128-byte swizzle
+  CUtensorMap map_p0;      // plane 0: N rows x K*b0/8 bytes, box 8*b0 x 128
+  CUtensorMap map_p1;      // plane 1 (widths 3, 6): box 16 bytes x 128
   const float* alpha;
   const float* zero;
   const float* sx;         // Sx[m] = sum_k x[m,k]
@@ -112,61 +114,54 @@ __device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// Unpacks 64 consecutive codes of one weight row into 32 bf16x2 registers
+// Unpacks 32 consecutive codes of one weight row into 16 bf16x2 registers
 // (register j holds codes 2j, 2j+1: the even code in the low half, as the
-// A operand in tensor memory expects). `p0` / `p1` point at this row's 64-code
+// A operand in tensor memory expects). `p0` / `p1` point at this row's 32-code
 // slice of plane 0 / plane 1 in shared memory. Plane word layout: local code
 // u of a width-b word sits at bit 16*(u%2) + b*(u/2) (b < 8), at 8u for b = 8.
 template <int R>
-__device__ __forceinline__ void decode64(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[32]) {
+__device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[16]) {
   if constexpr (R == 2) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p0);
+    const uint32_t w[2] = {a.x, a.y};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u);
+  } else if constexpr (R == 4) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u);
-  } else if constexpr (R == 4) {
-    const uint4 a = *reinterpret_cast<const uint4*>(p0);
-    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu);
+    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu);
   } else if constexpr (R == 3) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p0);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p1);
+    const uint32_t w[2] = {a.x, a.y};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t lo = (w[j / 8] >> (2 * (j % 8))) & 0x00030003u;
+      const uint32_t hi = ((u >> j) & 0x00010001u) << 2;
+      v[j] = exact_pair(lo | hi);
+    }
+  } else if constexpr (R == 6) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint2 h = *reinterpret_cast<const uint2*>(p1);
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
     const uint32_t u[2] = {h.x, h.y};
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t lo = (w[j / 8] >> (2 * (j % 8))) & 0x00030003u;
-      const uint32_t hi = ((u[j / 16] >> (j % 16)) & 0x00010001u) << 2;
-      v[j] = exact_pair(lo | hi);
-    }
-  } else if constexpr (R == 6) {
-    const uint4 a = *reinterpret_cast<const uint4*>(p0);
-    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
-    const uint4 h = *reinterpret_cast<const uint4*>(p1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    const uint32_t u[4] = {h.x, h.y, h.z, h.w};
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 16; ++j) {
       const uint32_t lo = (w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu;
       const uint32_t hi = ((u[j / 8] >> (2 * (j % 8))) & 0x00030003u) << 4;
       v[j] = exact_pair(lo | hi);
     }
   } else {  // R == 8: bytes, 4 codes per word
-    uint32_t w[16];
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 a = *reinterpret_cast<const uint4*>(p0 + 16 * i);
-      w[4 * i] = a.x; w[4 * i + 1] = a.y; w[4 * i + 2] = a.z; w[4 * i + 3] = a.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
+    for (int j = 0; j < 16; ++j)
       v[j] = (j % 2 == 0) ? exact_pair_bytes(w[j / 2], 0x7440u, 0x7441u)
                           : exact_pair_bytes(w[j / 2], 0x7442u, 0x7443u);
   }
 }
-
 
 // ------------------------------------------------------------ kernel
 template <int R>
@@ -216,8 +211,11 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       prefetch_tmap(&p.map_x);
       prefetch_tmap(&p.map_p0);
       int issued = 0;
-      const uint32_t p0_bytes = 128u * 16u * (R == 8 ? 8 : (R == 4 || R == 6) ? 4 : 2);
-      const uint32_t p1_bytes = (R == 3) ? 128u * 16u : (R == 6) ? 128u * 32u : 0u;
+      // plane 0: 8*b0 bytes (64 codes) per row; plane 1: the 16-byte chunk
+      // that holds the stage's codes (64 codes at b1 = 2, 128 at b1 = 1)
+      constexpr uint32_t b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
+      const uint32_t p0_bytes = 128u * 8u * b0;
+      const uint32_t p1_bytes = (R == 3 || R == 6) ? 128u * 16u : 0u;
       for (int it = 0; it < n_k; ++it, ++issued) {
         const int s = it % kStages;
         if (it >= kStages &&
@@ -230,9 +228,11 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
         mbar_arrive_expect_tx(&full[s], kXStageBytes + p0_bytes + p1_bytes);
         const int k0 = it * kBK;
         tma_load_2d(st, &p.map_x, k0, m0, &full[s]);
-        tma_load_2d(st + kXSubBytes, &p.map_x, k0 + 64, m0, &full[s]);
-        tma_load_2d(st + p.off_p0, &p.map_p0, it * static_cast<int>(p0_bytes / 128u), n0, &full[s]);
-        if (p1_bytes) tma_load_2d(st + p.off_p1, &p.map_p1, it * static_cast<int>(p1_bytes / 128u), n0, &full[s]);
+        tma_load_2d(st + p.off_p0, &p.map_p0, it * static_cast<int>(8 * b0), n0, &full[s]);
+        if (p1_bytes) {
+          const int x1 = (R == 3) ? (it / 2) * 16 : it * 16;
+          tma_load_2d(st + p.off_p1, &p.map_p1, x1, n0, &full[s]);
+        }
       }
       // no bulk copy may be in flight when this thread leaves
       const int first = issued > kStages ? issued - kStages : 0;
@@ -256,10 +256,10 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
         const uint32_t xs = smem_u32(stages + static_cast<size_t>(s) * p.stage_bytes);
 #pragma unroll
         for (int j = 0; j < kBK / 16; ++j) {
-          // k16 step j: A columns advance by 8 (two bf16 per column); B stays in
-          // sub-tile j / 4 and advances 32 bytes along its 128-byte rows.
-          const uint64_t bdesc = tc05::desc_kmajor_sw128(xs + (j / 4) * kXSubBytes + (j % 4) * 32);
-          tc05::mma_ts(tmem + kAccCol, tmem + kASlotCol + s * 64 + j * 8, bdesc, idesc,
+          // k16 step j: A columns advance by 8 (two bf16 per column); B advances
+          // 32 bytes along its 128-byte swizzled rows.
+          const uint64_t bdesc = tc05::desc_kmajor_sw128(xs + j * 32);
+          tc05::mma_ts(tmem + kAccCol, tmem + kASlotCol + s * 32 + j * 8, bdesc, idesc,
                        it > 0 || j > 0);
         }
         tc05::commit(smem_u32(&empty[s]));
@@ -272,7 +272,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
   } else if (warp >= kDecodeWarp0) {
     // ---------------------------------------------------------- decode
     const int q = warp & 3;                    // TMEM lane quarter of this warp
-    const int h = (warp - kDecodeWarp0) >> 2;  // which 64 codes of the stage
+    const int h = (warp - kDecodeWarp0) >> 2;  // which 32 codes of the stage
     const int row = 32 * q + lane;             // weight row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     constexpr int b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
@@ -291,18 +291,22 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
         break;
       }
       const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
-      const uint8_t* r0 = st + p.off_p0 + row * (16 * b0) + h * (8 * b0);
-      const uint8_t* r1 = st + p.off_p1 + row * (16 * (b1 ? b1 : 1)) + h * (8 * (b1 ? b1 : 1));
-      uint32_t v[32];
-      decode64<R>(r0, r1, v);
-      tc05::st_32x32b_x32(tmem + lane_addr + kASlotCol + s * 64 + h * 32, v);
+      // plane 0 rows hold 64 codes (8*b0 bytes); this warp's 32 codes are half
+      // of them. Plane 1 rows hold a 16-byte chunk: 64 codes at b1 = 2, 128 at
+      // b1 = 1 (of which this stage uses the half it % 2).
+      const uint8_t* r0 = st + p.off_p0 + row * (8 * b0) + h * (4 * b0);
+      const uint8_t* r1 = st + p.off_p1 + row * 16 +
+                          (b1 == 1 ? (it % 2) * 8 + h * 4 : h * 8);
+      uint32_t v[16];
+      decode32<R>(r0, r1, v);
+      tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&decoded[s]);
     }
     // ---------------------------------------------------------- epilogue
-    // Warp (q, h) writes batch columns [64 h, 64 h + 64) of its 32 weight rows.
+    // Warp (q, h) writes batch columns [128 h, 128 h + 128) of its 32 weight rows.
     const bool acc_ready = ok && __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0, p.wait_ns));
     if (acc_ready) {
       tc05::fence_after_sync();
@@ -315,8 +319,8 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
         B = a * __ldg(p.zero + n);
       }
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const int col = 64 * h + 32 * c;
+      for (int c = 0; c < 4; ++c) {
+        const int col = 128 * h + 32 * c;
         uint32_t d[32];
         tc05::ld_32x32b_x32(tmem + lane_addr + kAccCol + col, d);
         tc05::wait_ld();
@@ -378,11 +382,11 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, true);
   if (e != cudaSuccess) return e;
   e = encode_map_2d(&gp.map_p0, job.packed, uint64_t(job.N), uint64_t(job.K) * b0 / 8,
-                    16u * b0, kBN, 1);
+                    8u * b0, kBN, 1);
   if (e != cudaSuccess) return e;
   if (b1) {
     e = encode_map_2d(&gp.map_p1, job.packed + job.N * job.K * b0 / 8, uint64_t(job.N),
-                      uint64_t(job.K) * b1 / 8, 16u * b1, kBN, 1);
+                      uint64_t(job.K) * b1 / 8, 16u, kBN, 1);
     if (e != cudaSuccess) return e;
   } else {
     gp.map_p1 = gp.map_p0;
@@ -407,9 +411,9 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   gp.K = static_cast<int>(job.K);
   gp.r = job.r;
   gp.off_p0 = kXStageBytes;
-  const uint32_t p0_bytes = 128u * 16u * b0;
+  const uint32_t p0_bytes = 128u * 8u * b0;
   gp.off_p1 = gp.off_p0 + p0_bytes;
-  const uint32_t p1_bytes = 128u * 16u * b1;
+  const uint32_t p1_bytes = b1 ? 128u * 16u : 0u;
   gp.stage_bytes = (gp.off_p1 + p1_bytes + 1023u) & ~1023u;
   const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(kStages) * gp.stage_bytes;
 
