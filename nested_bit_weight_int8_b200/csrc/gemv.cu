@@ -123,13 +123,44 @@ constexpr uint32_t kMag4 = 0x40804080u, kMag8 = 0x41004100u, kMag16 = 0x41804180
 constexpr uint32_t kMaskP3b2 = 0x00180018u, kMaskP5b2 = 0x00600060u, kMaskP3b4 = 0x00780078u,
                    kMaskP0b4 = 0x000F000Fu;
 
+// bf16x2 a - b, exact here: both are small integers (magic + code, magic).
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// The pair of 2-bit codes at half-word position P (0, 2, ..., 14) of a plane
+// word as bf16x2. Positions 0-4 need no shift, 6-10 one shift by 6, 12-14 one
+// by 12, so a word costs two shifts and eight LOP3s. The code lands at bit
+// p = P mod 6 of each half, under the magic 2^(7-p) that gives it weight 1:
+// offsets 32 (p = 2) and 8 (p = 4) stay, and the 128 of p = 0 is subtracted
+// again at once on the FMA pipe, which keeps the fp32 sums small.
+template <int P>
+__device__ __forceinline__ uint32_t pick2(uint32_t w) {
+  constexpr int sh = P <= 4 ? 0 : (P <= 10 ? 6 : 12);
+  constexpr int p = P - sh;
+  constexpr uint32_t mask = 0x00030003u << p;
+  if constexpr (p == 0) {
+    return bf16x2_sub(and_or(w >> sh, mask, kMag128), kMag128);
+  } else {
+    return and_or(w >> sh, mask, p == 2 ? kMag32 : kMag8);
+  }
+}
+
 // Decoded A registers of one MMA for one weight row: x0 fills k-slots
 // {2t, 2t+1}, x1 fills {2t+8, 2t+9}. PLANE 0 is the low plane, 1 the high
 // plane; Q is the 8-code group of the chunk, HF the 4-code half of it.
 template <int R, int PLANE, int Q, int HF>
 __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint32_t (&hi)[2],
                                             uint32_t& x0, uint32_t& x1) {
-  if constexpr (R == 2 || (R == 3 && PLANE == 0)) {
+  if constexpr (R == 2) {
+    // 2-bit codes, word = 16 codes; x0 holds codes 4j, 4j+1 (half-word
+    // position 4j), x1 codes 4j+2, 4j+3 (position 4j+2), j = 2(Q%2)+HF.
+    constexpr int j = 2 * (Q % 2) + HF;
+    x0 = pick2<4 * j>(lo[Q / 2]);
+    x1 = pick2<4 * j + 2>(lo[Q / 2]);
+  } else if constexpr (R == 3 && PLANE == 0) {
     // 2-bit codes, word = 16 codes; pairs 2j, 2j+1 (j = 2(Q%2)+HF) at half-bits
     // 4j, 4j+2 -> bits 3-4 (16 + c) and bits 5-6 (4 + c) after one shift.
     constexpr int j = 2 * (Q % 2) + HF;
@@ -170,17 +201,16 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
 }
 
 // Offset of the decoded value per activation class (k >> 1) & 7 for each
-// width (the sum over the planes of the magic added to the code). The codes
-// sit in the top mantissa bits, so the offsets stay small next to the code
-// unit (16 or 4 at r = 2): the fp32 sums then lose little to cancellation when
-// the offsets are taken out again.
+// width (the sum over the planes of the magic added to the code). The offsets
+// stay small next to the code unit (at most 32 at r = 2), so the fp32 sums
+// lose little to cancellation when the offsets are taken out again.
 __device__ __forceinline__ void offset_coeffs(int r, float (&c)[kClasses]) {
-  constexpr float r2[4] = {16.f, 4.f, 16.f, 4.f};
+  constexpr float r2[kClasses] = {0.f, 32.f, 8.f, 0.f, 32.f, 8.f, 0.f, 32.f};
   constexpr float r3[4] = {80.f, 36.f, 32.f, 12.f};
   constexpr float r6[4] = {272.f, 80.f, 272.f, 80.f};
 #pragma unroll
   for (int i = 0; i < kClasses; ++i) {
-    c[i] = r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i & 3] : r == 3 ? r3[i & 3] : r6[i & 3];
+    c[i] = r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
   }
 }
 
@@ -193,10 +223,12 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[2][4], const uin
   uint4 xb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
+    // a plain shared-memory load (the CTA's dynamic shared array plus an
+    // offset), so the compiler may hoist it ahead of the decode work; the
+    // mbarrier wait before the unit is a memory barrier it cannot cross
+    extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t a = xaddr[nt] + static_cast<uint32_t>(gbase + Q) * xstep[nt];
-    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(xb[nt].x), "=r"(xb[nt].y), "=r"(xb[nt].z), "=r"(xb[nt].w)
-                 : "r"(a));
+    xb[nt] = *reinterpret_cast<const uint4*>(smem + a);
   }
   // two operand planes for r = 3, 6 (low/high bit planes) and r = 8 (low/high nibbles)
   constexpr int NPL = (Geo<R>::b1 != 0 || R == 8) ? 2 : 1;
@@ -366,7 +398,8 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
     }
     if (active) {
       const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
-      const uint32_t xs = smem_u32(st + p.off_x);
+      extern __shared__ __align__(128) uint8_t smem[];
+      const uint32_t xs = static_cast<uint32_t>(st + p.off_x - smem);  // offset in shared memory
       uint32_t xa[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) xa[nt] = xstep[nt] ? xs + xaddr[nt] : xaddr[nt];
@@ -375,7 +408,10 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
       for (int b = 0; b < NT; ++b)
 #pragma unroll
         for (int j = 0; j < 4; ++j) { ch[b][0][j] = 0.f; ch[b][1][j] = 0.f; }
-      process_unit<R, NT, NSUB>(st, st + p.off_plane1, xa, xstep, p.pitch0, p.pitch1, warp, lane,
+      // The plane pitches follow from the batch tiles (the host picks 192
+      // bytes per row for M <= 8, 64 otherwise), so they are compile-time here.
+      constexpr int kP0 = (NT == 1) ? 192 : 64;
+      process_unit<R, NT, NSUB>(st, st + kRowsPerUnit * kP0, xa, xstep, kP0, kP0 / 2, warp, lane,
                                 ch);
 #pragma unroll
       for (int b = 0; b < NT; ++b)
@@ -483,7 +519,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   pdl_wait_primary();
   const int g = lane >> 2, t = lane & 3;
   uint32_t xaddr[NT], xstep[NT];
-  const uint32_t zero_addr = smem_u32(zero_block) + t * 16;
+  const uint32_t zero_addr = static_cast<uint32_t>(zero_block - smem) + t * 16;  // shared offset
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int m = nt * 8 + g;
