@@ -19,7 +19,8 @@
 // stay below the MMA time of a stage.
 //   warp 0      : TMA producer (x box, plane boxes) into a ring of stages
 //   warp 1      : allocates tensor memory, issues tcgen05.mma (one thread)
-//   warps 4..11 : decode: each thread owns one weight row (its TMEM lane) and
+//   warps 4..19 : decode, two groups of eight taking alternate stages: each
+//                 thread owns one weight row (its TMEM lane) and
 //                 32 of the stage's 64 codes, unpacks them from the staged
 //                 planes to bf16 and writes them to tensor memory
 //                 (tcgen05.st); then the same warps run the epilogue.
@@ -45,8 +46,8 @@ constexpr int kBN = 128;          // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int kBM = 256;          // batch rows per CTA (MMA N, TMEM columns)
 constexpr int kBK = 64;           // codes of K per stage
 constexpr int kStages = 5;
-constexpr int kGemmThreads = 12 * 32;
-constexpr int kDecodeWarp0 = 4;   // warps 4..11 decode, then run the epilogue
+constexpr int kGemmThreads = 20 * 32;
+constexpr int kDecodeWarp0 = 4;   // warps 4..19 decode, then run the epilogue
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                 // D: columns [0, 256)
 constexpr uint32_t kASlotCol = 256;             // A slot s: columns [256 + 32 s, +32)
@@ -183,7 +184,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
   const int n_k = p.K / kBK;
-  constexpr int kDecodeWarps = 8;
+  constexpr int kDecodeWarps = 8;   // per stage: one of the two decode groups
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -271,14 +272,18 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
     }
   } else if (warp >= kDecodeWarp0) {
     // ---------------------------------------------------------- decode
-    const int q = warp & 3;                    // TMEM lane quarter of this warp
-    const int h = (warp - kDecodeWarp0) >> 2;  // which 32 codes of the stage
+    // Two groups of eight warps take alternate stages: the decode of a stage
+    // is a chain of waits and a tensor-memory store whose latency exceeds the
+    // MMA time of one stage, so each group gets two stages' time for it.
+    const int q = warp & 3;                          // TMEM lane quarter of this warp
+    const int h = ((warp - kDecodeWarp0) >> 2) & 1;  // which 32 codes of the stage
+    const int grp = (warp - kDecodeWarp0) >> 3;      // which stages: it % 2 == grp
     const int row = 32 * q + lane;             // weight row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     constexpr int b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
     constexpr int b1 = (R == 3) ? 1 : (R == 6) ? 2 : 0;
     bool ok = true;
-    for (int it = 0; it < n_k; ++it) {
+    for (int it = grp; it < n_k; it += 2) {
       const int s = it % kStages;
       // Every lane waits (each needs the barrier's ordering for the staged
       // bytes); the warp then decides together, since the tensor-memory
@@ -306,7 +311,8 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       if (lane == 0) mbar_arrive(&decoded[s]);
     }
     // ---------------------------------------------------------- epilogue
-    // Warp (q, h) writes batch columns [128 h, 128 h + 128) of its 32 weight rows.
+    // Warp (q, h, grp) writes batch columns [128 h + 64 grp, +64) of its 32
+    // weight rows.
     const bool acc_ready = ok && __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0, p.wait_ns));
     if (acc_ready) {
       tc05::fence_after_sync();
@@ -319,8 +325,8 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
         B = a * __ldg(p.zero + n);
       }
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int col = 128 * h + 32 * c;
+      for (int c = 0; c < 2; ++c) {
+        const int col = 128 * h + 64 * grp + 32 * c;
         uint32_t d[32];
         tc05::ld_32x32b_x32(tmem + lane_addr + kAccCol + col, d);
         tc05::wait_ld();
