@@ -408,7 +408,7 @@ def run_gpu(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 x int-code planes, fp32 accumulate",
+        "dtype": "bf16",
         "data": "synthetic (seeded torch normal weights N(0,0.02^2), activations N(0,1))",
         "config": {
             "workload": WORKLOAD,
@@ -418,6 +418,7 @@ def run_gpu(args, rank, world, local):
             "M": args.M,
             "linears": len(stack.lins),
             "packed_bytes_per_step": stack.packed_bytes,
+            "arithmetic": "bf16 activations x exact integer codes (bf16), fp32 accumulate",
             "l2": "inputs larger than L2: 3.49 GB of packed planes streamed per step",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
