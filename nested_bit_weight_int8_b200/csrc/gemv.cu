@@ -48,16 +48,32 @@ namespace mq {
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kTilesPerWarp = 1;
-constexpr int kRowsPerWarp = 16 * kTilesPerWarp;
-constexpr int kRowsPerUnit = kConsumerWarps * kTilesPerWarp * 16;  // 128
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxStages = 8;
-constexpr int kBarrierBytes = 256;  // barriers, abort flag; last 64 bytes: zero block
+constexpr int kHeaderBytes = 1024;  // barriers, abort flag; last 64 bytes: zero block
 constexpr int kMaxDynSmem = 227 * 1024;
-constexpr size_t kStageBudget = 110 * 1024;
+constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header and alignment slack
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
 constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
+
+// Geometry of a launch with NT batch tiles of 8. Up to 8 batch rows, each
+// consumer warp owns two 16-row tiles (four independent MMA chains; one
+// activation fragment load feeds two MMAs) over 128-byte plane rows staged in
+// 128-byte swizzled boxes, so a unit is 256 rows. Larger batches keep one
+// tile per warp over 64-byte rows (128-row units): their accumulators take
+// the registers.
+template <int NT>
+struct Tiling {
+  static constexpr int TW = (NT == 1) ? 2 : 1;       // 16-row tiles per warp
+  static constexpr int RPW = 16 * TW;                // weight rows per warp
+  static constexpr int RPU = kConsumerWarps * RPW;   // weight rows per unit
+  static constexpr int P0 = (NT == 1) ? 128 : 64;    // plane-0 bytes per row per unit
+  static constexpr bool SWZ = (NT == 1);             // plane-0 box in 128-byte swizzle
+  static constexpr int NSUB = P0 / 64;               // 64-byte sub-steps per unit
+};
+// The same choice on the host, by batch size.
+inline int tiling_p0(int M) { return M <= 8 ? 128 : 64; }
+inline int tiling_rows(int M) { return M <= 8 ? 256 : 128; }
 
 // Per-linear descriptor, passed by value in the kernel parameters.
 struct LinDesc {
@@ -216,10 +232,10 @@ __device__ __forceinline__ void offset_coeffs(int r, float (&c)[kClasses]) {
 
 // All MMAs of one 8-code activation group: for each 4-code half and each
 // plane, one m16n8k16 per batch tile, the B registers shared by the planes.
-template <int R, int NT, int Q>
-__device__ __forceinline__ void group_mmas(const uint32_t (&lo)[2][4], const uint32_t (&hi)[2][2],
+template <int R, int NT, int TW, int Q>
+__device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, float (&ch)[NT][2][4]) {
+                                           int gbase, float (&ch)[TW][NT][2][4]) {
   uint4 xb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -236,64 +252,74 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[2][4], const uin
   for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
     for (int pl = 0; pl < NPL; ++pl) {
-      uint32_t a0, a1, a2, a3;
-      if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[0], hi[0], a0, a2); decode_quad<R, 0, Q, 0>(lo[1], hi[1], a1, a3); }
-      if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[0], hi[0], a0, a2); decode_quad<R, 1, Q, 0>(lo[1], hi[1], a1, a3); }
-      if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[0], hi[0], a0, a2); decode_quad<R, 0, Q, 1>(lo[1], hi[1], a1, a3); }
-      if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[0], hi[0], a0, a2); decode_quad<R, 1, Q, 1>(lo[1], hi[1], a1, a3); }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t b0 = hf ? xb[nt].z : xb[nt].x;
-        const uint32_t b1 = hf ? xb[nt].w : xb[nt].y;
-        mma_bf16_16816(ch[nt][(2 * Q + hf + pl) & 1], a0, a1, a2, a3, b0, b1);
+      for (int T = 0; T < TW; ++T) {
+        uint32_t a0, a1, a2, a3;
+        if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 0, Q, 0>(lo[T][1], hi[T][1], a1, a3); }
+        if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 1, Q, 0>(lo[T][1], hi[T][1], a1, a3); }
+        if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 0, Q, 1>(lo[T][1], hi[T][1], a1, a3); }
+        if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 1, Q, 1>(lo[T][1], hi[T][1], a1, a3); }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint32_t b0 = hf ? xb[nt].z : xb[nt].x;
+          const uint32_t b1 = hf ? xb[nt].w : xb[nt].y;
+          mma_bf16_16816(ch[T][nt][(2 * Q + hf + pl) & 1], a0, a1, a2, a3, b0, b1);
+        }
       }
     }
   }
 }
 
-template <int R, int NT, int... Qs>
-__device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[2][4], const uint32_t (&hi)[2][2],
+template <int R, int NT, int TW, int... Qs>
+__device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, float (&ch)[NT][2][4],
+                                           int gbase, float (&ch)[TW][NT][2][4],
                                            std::integer_sequence<int, Qs...>) {
-  (group_mmas<R, NT, Qs>(lo, hi, xaddr, xstep, gbase, ch), ...);
+  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, ch), ...);
 }
 
-// One staged unit for this warp's 16-row tile. All NSUB sub-steps are
-// unrolled and their plane loads issued first. Sub-steps past the unit's
-// valid codes read zero-filled planes and zero activations and add nothing.
-// Activation group q of chunk 4s+t for batch row m sits at
-// ((((s*W8 + q)*M + m)*4 + t) * 16) bytes of the staged block; lanes whose
-// batch row is past M read a zero block instead (step 0).
-template <int R, int NT, int NSUB>
+// One staged unit for this warp's 16-row tiles. All sub-steps are unrolled
+// and their plane loads issued first. Sub-steps past the unit's valid codes
+// read zero-filled planes and zero activations and add nothing. Activation
+// group q of chunk 4s+t for batch row m sits at ((((s*W8 + q)*M + m)*4 + t)
+// * 16) bytes of the staged block; lanes whose batch row is past M read a
+// zero block instead (step 0). With 128-byte plane rows the box is stored in
+// 128-byte swizzled atoms: chunk c of row r at chunk c ^ (r % 8).
+template <int R, int NT>
 __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* st1,
                                              const uint32_t (&xaddr)[NT],
-                                             const uint32_t (&xstep)[NT], int pitch0, int pitch1,
-                                             int warp, int lane, float (&ch)[NT][2][4]) {
+                                             const uint32_t (&xstep)[NT], int warp, int lane,
+                                             float (&ch)[Tiling<NT>::TW][NT][2][4]) {
   using G = Geo<R>;
+  using TL = Tiling<NT>;
+  constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0, P1 = TL::P0 / 2;
   const int g = lane >> 2, t = lane & 3;
-  uint32_t lo[NSUB][2][4];
-  uint32_t hi[NSUB][2][2];
+  uint32_t lo[NSUB][TW][2][4];
+  uint32_t hi[NSUB][TW][2][2];
 #pragma unroll
   for (int s = 0; s < NSUB; ++s) {
     const int ci = 4 * s + t;  // this thread's 16-byte chunk of the low plane
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = warp * kRowsPerWarp + g + 8 * h;
-      const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * pitch0 + ci * 16);
-      lo[s][h][0] = v.x; lo[s][h][1] = v.y; lo[s][h][2] = v.z; lo[s][h][3] = v.w;
-      if constexpr (G::b1 != 0) {
-        const uint2 u = *reinterpret_cast<const uint2*>(st1 + row * pitch1 + ci * 8);
-        hi[s][h][0] = u.x; hi[s][h][1] = u.y;
-      } else {
-        hi[s][h][0] = 0; hi[s][h][1] = 0;
+    for (int T = 0; T < TW; ++T) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = warp * TL::RPW + 16 * T + g + 8 * h;
+        const int cs = TL::SWZ ? (ci ^ (row & 7)) : ci;
+        const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * P0 + cs * 16);
+        lo[s][T][h][0] = v.x; lo[s][T][h][1] = v.y; lo[s][T][h][2] = v.z; lo[s][T][h][3] = v.w;
+        if constexpr (G::b1 != 0) {
+          const uint2 u = *reinterpret_cast<const uint2*>(st1 + row * P1 + ci * 8);
+          hi[s][T][h][0] = u.x; hi[s][T][h][1] = u.y;
+        } else {
+          hi[s][T][h][0] = 0; hi[s][T][h][1] = 0;
+        }
       }
     }
   }
 #pragma unroll
   for (int s = 0; s < NSUB; ++s)
-    chunk_mmas<R, NT>(lo[s], hi[s], xaddr, xstep, s * G::W8, ch,
-                      std::make_integer_sequence<int, G::W8>{});
+    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, ch,
+                          std::make_integer_sequence<int, G::W8>{});
 }
 
 // The current linear of a CTA's walk over its unit range, cached in registers.
@@ -302,34 +328,34 @@ struct Cursor {
   int nrb, n_kc, r, N;    // of linear l
 };
 
-template <int CAP>
+template <int RPU, int CAP>
 __device__ __forceinline__ void cursor_load(const GemvParams<CAP>& p, Cursor& c) {
   const LinDesc& L = p.lin[c.l];
   c.n_kc = L.n_kc;
-  c.nrb = (L.N + kRowsPerUnit - 1) / kRowsPerUnit;
+  c.nrb = (L.N + RPU - 1) / RPU;
   c.r = L.r;
   c.N = L.N;
 }
 
-template <int CAP>
+template <int RPU, int CAP>
 __device__ __forceinline__ void cursor_init(const GemvParams<CAP>& p, int u, Cursor& c) {
   int l = 0;
   while (l + 1 < p.n_lin && u >= p.lin[l + 1].unit_begin) ++l;
   c.l = l;
-  cursor_load(p, c);
+  cursor_load<RPU>(p, c);
   const int local = u - p.lin[l].unit_begin;
   c.rb = local / c.n_kc;
   c.kc = local - c.rb * c.n_kc;
 }
 
-template <int CAP>
+template <int RPU, int CAP>
 __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c) {
   if (++c.kc == c.n_kc) {
     c.kc = 0;
     if (++c.rb == c.nrb) {
       c.rb = 0;
       ++c.l;
-      if (c.l < p.n_lin) cursor_load(p, c);
+      if (c.l < p.n_lin) cursor_load<RPU>(p, c);
     }
   }
 }
@@ -341,7 +367,7 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
 // zeroed.
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
-                           int lane, const float (&tot)[NT][4]) {
+                           int T, int lane, const float (&tot)[NT][4]) {
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
@@ -349,7 +375,7 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
   offset_coeffs(L.r, c);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int n = rb * kRowsPerUnit + warp * kRowsPerWarp + g + 8 * h;
+    const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h;
     if (n >= L.N) continue;
     const float a = L.alpha[n], z = L.zero[n];
     const float A = a * scale, B = a * z;
@@ -384,13 +410,14 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
 // adds them into `tot`. The two MMA accumulator chains are folded into `tot`
 // after every unit, which keeps each fp32 chain short. Returns false if a wait
 // gave up (the abort flag is then set for the whole CTA).
-template <int R, int NT, int NSUB, int CAP>
+template <int R, int NT, int CAP>
 __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint8_t* stages,
                                             uint64_t* full, uint64_t* empty,
                                             volatile int* s_abort, int seg, int& s, uint32_t& ph,
                                             bool active, const uint32_t (&xaddr)[NT],
                                             const uint32_t (&xstep)[NT], int warp, int lane,
-                                            float (&tot)[NT][4]) {
+                                            float (&tot)[Tiling<NT>::TW][NT][4]) {
+  constexpr int TW = Tiling<NT>::TW;
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
       if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
@@ -403,20 +430,21 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
       uint32_t xa[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) xa[nt] = xstep[nt] ? xs + xaddr[nt] : xaddr[nt];
-      float ch[NT][2][4];
+      float ch[TW][NT][2][4];
 #pragma unroll
-      for (int b = 0; b < NT; ++b)
+      for (int T = 0; T < TW; ++T)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) { ch[b][0][j] = 0.f; ch[b][1][j] = 0.f; }
-      // The plane pitches follow from the batch tiles (the host picks 192
-      // bytes per row for M <= 8, 64 otherwise), so they are compile-time here.
-      constexpr int kP0 = (NT == 1) ? 192 : 64;
-      process_unit<R, NT, NSUB>(st, st + kRowsPerUnit * kP0, xa, xstep, kP0, kP0 / 2, warp, lane,
-                                ch);
+        for (int b = 0; b < NT; ++b)
 #pragma unroll
-      for (int b = 0; b < NT; ++b)
+          for (int j = 0; j < 4; ++j) { ch[T][b][0][j] = 0.f; ch[T][b][1][j] = 0.f; }
+      // the plane pitches and rows follow from the batch tiles (Tiling)
+      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, ch);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tot[b][j] += ch[b][0][j] + ch[b][1][j];
+      for (int T = 0; T < TW; ++T)
+#pragma unroll
+        for (int b = 0; b < NT; ++b)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tot[T][b][j] += ch[T][b][0][j] + ch[T][b][1][j];
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -428,12 +456,16 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
 template <int NT, int CAP>
 __global__ void __launch_bounds__(kGemvThreads, (NT <= 2 ? 2 : 1))
 gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
+  using TL = Tiling<NT>;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  // 1024-byte aligned header and stages: the swizzled plane boxes need it
+  const uint32_t raw = smem_u32(smem);
+  uint8_t* base = smem + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base);
   uint64_t* empty = full + kMaxStages;
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
-  uint8_t* zero_block = smem + kBarrierBytes - 64;  // 64 zero bytes read by lanes past M
-  uint8_t* stages = smem + kBarrierBytes;
+  uint8_t* zero_block = base + kHeaderBytes - 64;  // 64 zero bytes read by lanes past M
+  uint8_t* stages = base + kHeaderBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
 
@@ -461,20 +493,20 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
     int issued = 0;
     if (lane == 0) {
       Cursor c;
-      cursor_init(p, u0, c);
+      cursor_init<TL::RPU>(p, u0, c);
       Cursor pre_c = c;
       auto issue_weights = [&](const Cursor& cc, int s) {
         int b0, b1;
         plane_widths_dev(cc.r, b0, b1);
         uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
         const CUtensorMap* tm = p.map_table ? p.map_table + 2 * cc.l : &p.maps[2 * cc.l];
-        const uint32_t box = kRowsPerUnit * (p.pitch0 + (b1 ? p.pitch1 : 0));
+        const uint32_t box = TL::RPU * (p.pitch0 + (b1 ? p.pitch1 : 0));
         const uint32_t bytesx = static_cast<uint32_t>(p.M * p.lin[cc.l].kc * 2);
         // One 2-D box per plane (128 rows x the unit's bytes; rows past N and
         // bytes past K read as zero) plus the unit's activation block.
         mbar_arrive_expect_tx(&full[s], box + bytesx);
-        tma_load_2d(st, tm, cc.kc * p.pitch0, cc.rb * kRowsPerUnit, &full[s]);
-        if (b1) tma_load_2d(st + p.off_plane1, tm + 1, cc.kc * p.pitch1, cc.rb * kRowsPerUnit, &full[s]);
+        tma_load_2d(st, tm, cc.kc * p.pitch0, cc.rb * TL::RPU, &full[s]);
+        if (b1) tma_load_2d(st + p.off_plane1, tm + 1, cc.kc * p.pitch1, cc.rb * TL::RPU, &full[s]);
       };
       auto issue_x = [&](const Cursor& cc, int s) {
         const LinDesc& L = p.lin[cc.l];
@@ -483,9 +515,9 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         bulk_g2s(st + p.off_x, L.xf + int64_t(cc.kc) * bytesx, bytesx, &full[s]);
       };
       const int pre = min(S, u1 - u0);
-      for (int i = 0; i < pre; ++i) { issue_weights(c, i); cursor_next(p, c); }
+      for (int i = 0; i < pre; ++i) { issue_weights(c, i); cursor_next<TL::RPU>(p, c); }
       pdl_wait_primary();
-      for (int i = 0; i < pre; ++i) { issue_x(pre_c, i); cursor_next(p, pre_c); }
+      for (int i = 0; i < pre; ++i) { issue_x(pre_c, i); cursor_next<TL::RPU>(p, pre_c); }
       issued = pre;
       for (int u = u0 + pre; u < u1; ++u, ++issued) {
         const int s = issued % S;
@@ -498,7 +530,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         if (*s_abort) { aborted = true; break; }
         issue_weights(c, s);
         issue_x(c, s);
-        cursor_next(p, c);
+        cursor_next<TL::RPU>(p, c);
       }
       // Leave no bulk copy in flight when this thread exits, whether or not
       // the consumers took the data (they stop early after a wait gave up):
@@ -530,11 +562,8 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       xstep[nt] = static_cast<uint32_t>(p.M) * 64u;
     }
   }
-  // Sub-steps per unit: the low plane holds 192 bytes per row per unit for
-  // M <= 8 (3 sub-steps of 64 bytes) and 64 bytes for larger M.
-  constexpr int NSUB = (NT == 1) ? 3 : 1;
   Cursor c;
-  cursor_init(p, u0, c);
+  cursor_init<TL::RPU>(p, u0, c);
   int s = 0;
   uint32_t ph = 0;
   for (int u = u0; u < u1;) {
@@ -542,29 +571,34 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
     const int seg = min(c.n_kc - c.kc, u1 - u);
     const int kc0 = c.kc;
     const bool whole = kc0 == 0 && seg == c.n_kc;
-    const bool active = warp * kRowsPerWarp < c.N - c.rb * kRowsPerUnit;
-    float tot[NT][4];
+    const bool active = warp * TL::RPW < c.N - c.rb * TL::RPU;
+    float tot[TL::TW][NT][4];
 #pragma unroll
-    for (int b = 0; b < NT; ++b)
+    for (int T = 0; T < TL::TW; ++T)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tot[b][i] = 0.f;
+      for (int b = 0; b < NT; ++b)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tot[T][b][i] = 0.f;
     bool ok;
     switch (c.r) {
-      case 2: ok = run_segment<2, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 4: ok = run_segment<4, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 8: ok = run_segment<8, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 3: ok = run_segment<3, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      default: ok = run_segment<6, NT, NSUB>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+      default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
     }
     if (!ok) break;  // outputs are undefined after a give-up; the flag says so
-    if (active) flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot);
+    if (active) {
+#pragma unroll
+      for (int T = 0; T < TL::TW; ++T) flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, T, lane, tot[T]);
+    }
     u += seg;
     c.kc += seg;
     if (c.kc == c.n_kc) {
       c.kc = 0;
       if (++c.rb == c.nrb) {
         c.rb = 0;
-        if (++c.l < p.n_lin) cursor_load(p, c);
+        if (++c.l < p.n_lin) cursor_load<TL::RPU>(p, c);
       }
     }
   }
@@ -591,6 +625,7 @@ struct PrepZero {
 template <int CAP>
 struct PrepParams {
   int M, n_layout, n_sum, n_zero;
+  int rows;  // weight rows per unit: the height of a zeroed row block
   PrepLayout lay[CAP];
   PrepSum sum[CAP];
   PrepZero zero[kMaxCtas];
@@ -664,12 +699,12 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
     }
   }
   // (3) zero the shared output row blocks
-  const int64_t zt = int64_t(p.n_zero) * M * kRowsPerUnit;
+  const int64_t zt = int64_t(p.n_zero) * M * p.rows;
   for (int64_t i = tid; i < zt; i += stride) {
-    const PrepZero& Z = p.zero[i / (int64_t(M) * kRowsPerUnit)];
-    const int rem = static_cast<int>(i % (int64_t(M) * kRowsPerUnit));
-    const int m = rem / kRowsPerUnit;
-    const int n = Z.rb * kRowsPerUnit + rem % kRowsPerUnit;
+    const PrepZero& Z = p.zero[i / (int64_t(M) * p.rows)];
+    const int rem = static_cast<int>(i % (int64_t(M) * p.rows));
+    const int m = rem / p.rows;
+    const int n = Z.rb * p.rows + rem % p.rows;
     if (n < Z.N) Z.y[int64_t(m) * Z.N + n] = 0.f;
   }
 }
@@ -740,11 +775,13 @@ std::map<std::pair<int, std::vector<uint64_t>>, CUtensorMap*> g_map_tables;
 cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
   int b0, b1;
   plane_widths(j.r, b0, b1);
+  // 128-byte plane-0 rows go with 256-row units and the 128-byte swizzle
+  const uint32_t rows = P0 == 128 ? 256u : 128u;
   cudaError_t e = encode_map_2d(&out2[0], j.packed, uint64_t(j.N), uint64_t(j.K) * b0 / 8,
-                                static_cast<uint32_t>(P0), kRowsPerUnit, 1);
+                                static_cast<uint32_t>(P0), rows, 1, P0 == 128);
   if (e != cudaSuccess || !b1) return e;
   return encode_map_2d(&out2[1], j.packed + j.N * j.K * b0 / 8, uint64_t(j.N),
-                       uint64_t(j.K) * b1 / 8, static_cast<uint32_t>(P0 / 2), kRowsPerUnit, 1);
+                       uint64_t(j.K) * b1 / 8, static_cast<uint32_t>(P0 / 2), rows, 1);
 }
 
 cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUtensorMap** out) {
@@ -801,10 +838,10 @@ int64_t unit_cost(int r) {
 template <int CAP>
 cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream,
                          const FixedScratch* fixed = nullptr) {
-  // Bytes of low plane per row per unit: 192 keeps consecutive rows 64 bytes
-  // apart modulo 128 (conflict-free 16-byte shared loads) with few copies;
-  // larger batches use 64 to bound the staged activation block.
-  const int P0 = M <= 8 ? 192 : 64;
+  // Plane-0 bytes per row per unit and rows per unit (Tiling): 128 bytes in
+  // 256-row units up to 8 batch rows, 64 bytes in 128-row units above.
+  const int P0 = tiling_p0(M);
+  const int RU = tiling_rows(M);
   const int NT = (M + 7) / 8;
 
   static thread_local GemvParams<CAP> gp;
@@ -840,7 +877,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
       xf_bytes = (xf_bytes + 255) & ~size_t(255);
     }
     lay_of[i] = li;
-    const int nrb = static_cast<int>((j.N + kRowsPerUnit - 1) / kRowsPerUnit);
+    const int nrb = static_cast<int>((j.N + RU - 1) / RU);
     LinDesc& d = gp.lin[i];
     d.plane0 = j.packed;
     d.plane1 = b1 ? j.packed + j.N * j.K * b0 / 8 : nullptr;
@@ -885,14 +922,14 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
 
   // Stage layout: [128 rows x P0][128 rows x P1][M x KC bf16 activations].
   const int P1 = two_planes ? P0 / 2 : 0;
-  const uint32_t off_plane1 = static_cast<uint32_t>(kRowsPerUnit * P0);
-  const uint32_t off_x = off_plane1 + static_cast<uint32_t>(kRowsPerUnit * P1);
+  const uint32_t off_plane1 = static_cast<uint32_t>(RU * P0);
+  const uint32_t off_x = off_plane1 + static_cast<uint32_t>(RU * P1);
   const uint32_t x_bytes = static_cast<uint32_t>(M * (P0 * 8 / 2) * 2);  // largest KC (b0 = 2)
   uint32_t stage_bytes = off_x + x_bytes;
-  stage_bytes = (stage_bytes + 127) & ~127u;
+  stage_bytes = (stage_bytes + 1023) & ~1023u;  // swizzled boxes start 1024-aligned
   int stages = static_cast<int>(kStageBudget / stage_bytes);
   stages = std::max(2, std::min(stages, kMaxStages));
-  const size_t smem = kBarrierBytes + size_t(stages) * stage_bytes;
+  const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(stages) * stage_bytes;
   const int sms = sm_count();
   int grid = 1;
   switch (NT) {
@@ -950,6 +987,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   pp.n_layout = n_layouts;
   pp.n_sum = n_sums;
   pp.n_zero = n_zero;
+  pp.rows = RU;
   for (int i = 0; i < n_layouts; ++i) {
     pp.lay[i] = {static_cast<const __nv_bfloat16*>(layouts[i].x), wsb + layouts[i].off,
                  layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc,
@@ -1003,7 +1041,7 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
 
 size_t gemv_scratch_bytes(const LinearJob& job, int M) {
   // Same arithmetic as the planner in run_gemv_cap for one linear.
-  const int P0 = M <= 8 ? 192 : 64;
+  const int P0 = tiling_p0(M);
   int b0, b1;
   plane_widths(job.r, b0, b1);
   const int kc = P0 * 8 / b0;
