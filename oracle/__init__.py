@@ -8,6 +8,8 @@ Only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 It shares no code with the CUDA path. Everything here is float64 numpy or
 Python integers, written from the Matryoshka Quantization pages:
 
+* ``omniquant`` -- Eq. 3, OmniQuant's clipped MinMax with given per-row
+                  clipping factors gamma and beta (same page, section 3.4).
 * ``minmax``   -- Eq. 1, per-output-channel asymmetric MinMax int8 container
                   (page "Matryoshka Quantization" explainer, section 3.4,
                   "Quantization Primitives", Eq. 1; dequantization alpha*(q - z)).
@@ -25,12 +27,13 @@ Parity status: every function is pinned by tests under ``tests/`` that check
 it against values the pages print, closed forms, invariants or brute force.
 """
 from .minmax import quantize_minmax, dequantize, FP32_CONTRACT
+from .omniquant import quantize_omniquant
 from .slicing import slice_code, slice_value, slice_codes, slice_table
 from .planes import plane_widths, pack_rows, unpack_rows, packed_bytes, pack_rows_bigint
 from .matmul import dequant_slice, linear, tolerance, stack_forward
 
 __all__ = [
-    "quantize_minmax", "dequantize", "FP32_CONTRACT",
+    "quantize_minmax", "dequantize", "FP32_CONTRACT", "quantize_omniquant",
     "slice_code", "slice_value", "slice_codes", "slice_table",
     "plane_widths", "pack_rows", "unpack_rows", "packed_bytes", "pack_rows_bigint",
     "dequant_slice", "linear", "tolerance", "stack_forward",
