@@ -240,7 +240,7 @@ def time_device(fn, steps: int, warmup: int, stream, world: int, dev):
 
 def rows_timings(dev, stream):
     """Separately timed rows of the path on one 14336x4096 bf16 weight:
-    quantize (Eq. 1), slice-pack (Eq. 6) per width, one decode linear per
+    quantize (Eq. 1 and Eq. 3's clipped variant), slice-pack (Eq. 6) per width, one decode linear per
     width (M = 1), and the prefill GEMM at M = 2048 when served."""
     import torch
     import nested_bit_weight_int8_b200 as mq
@@ -274,6 +274,15 @@ def rows_timings(dev, stream):
     out = {}
     us = timed(lambda: mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z, stream))
     out["quantize_int8_14336x4096"] = {"us": round(us, 2), "GBps": round((n * k * 3 + 8 * n) / us / 1e3, 1)}
+    # Eq. 3 clipped variant, per-row gamma, beta in [0.6, 1]
+    gam = 0.6 + 0.4 * torch.rand(n, generator=gen, device=dev)
+    bet = 0.6 + 0.4 * torch.rand(n, generator=gen, device=dev)
+    qc = torch.empty_like(q)
+    us = timed(lambda: mq.quantize_int8_clipped(w, mq.MQ_BF16, n, k, gam, bet, qc, a, z, stream))
+    out["quantize_int8_clipped_14336x4096"] = {"us": round(us, 2),
+                                               "GBps": round((n * k * 3 + 16 * n) / us / 1e3, 1)}
+    mq.quantize_int8(w, mq.MQ_BF16, n, k, q, a, z, stream)
+    del qc
     x = torch.randn((1, k), generator=gen, device=dev).to(torch.bfloat16)
     y = torch.empty((1, n), dtype=torch.float32, device=dev)
     for r in (8, 4, 2):

@@ -94,6 +94,24 @@ MQ_API mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K
                            uint8_t* q, float* alpha, float* zero, void* stream);
 
 /*
+ * Eq. 3, OmniQuant's clipped MinMax quantization into the int8 container,
+ * with the clipping factors given (learning them is training, not serving):
+ *   alpha_n = (gamma_n * max_k w[n,k] - beta_n * min_k w[n,k]) / 255,
+ *   z_n     = -(beta_n * min_k w[n,k]) / alpha_n,
+ *   q[n,k]  = clamp(round(w[n,k] / alpha_n + z_n), 0, 255),
+ * so weights outside [beta_n min, gamma_n max] saturate at 0 or 255. Same
+ * arithmetic contract as mq_quantize_int8, with gmax = gamma * max and
+ * bmin = beta * min rounded first; a row whose clipped range is empty or
+ * inverted (alpha <= 0) gets alpha = 1 and z = -bmin. gamma = beta = 1 gives
+ * exactly mq_quantize_int8.
+ *   gamma, beta : N fp32 (device), 4-byte aligned, finite (OmniQuant keeps
+ *                 them in (0, 1)). Other arguments as mq_quantize_int8.
+ */
+MQ_API mq_status mq_quantize_int8_clipped(const void* w, int dtype, int64_t N, int64_t K,
+                                          const float* gamma, const float* beta, uint8_t* q,
+                                          float* alpha, float* zero, void* stream);
+
+/*
  * Eq. 6 slicing of the container into width r, packed as dense r-bit planes:
  *   code[n,k] = clamp(round_half_up(q[n,k] / 2^(8-r)), 0, 2^r - 1)
  * (S(q, r) = code * 2^(8-r); r = 8 is the identity). The first dropped bit

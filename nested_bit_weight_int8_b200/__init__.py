@@ -47,6 +47,8 @@ _version = _sig("mq_version", _int, [])
 _last_error = _sig("mq_last_error", ctypes.c_char_p, [])
 _packed_bytes = _sig("mq_packed_bytes", ctypes.c_size_t, [_i64, _i64, _int])
 _quantize = _sig("mq_quantize_int8", _int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp])
+_quantize_clipped = _sig("mq_quantize_int8_clipped", _int,
+                        [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp])
 _slice_pack = _sig("mq_slice_pack", _int, [_vp, _i64, _i64, _int, _vp, _vp])
 _linear = _sig("mq_linear", _int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
 _stack = _sig("mq_stack_forward", _int,
@@ -60,7 +62,8 @@ _wait_limit = _sig("mq_debug_set_wait_limit_ns", _int, [_u64])
 
 EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8",
             "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
-            "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc")
+            "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc",
+            "mq_quantize_int8_clipped")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -107,6 +110,13 @@ def packed_bytes(N: int, K: int, r: int) -> int:
 def quantize_int8(w, dtype: int, N: int, K: int, q, alpha, zero, stream=None) -> None:
     """Eq. 1 per-row MinMax int8 container: q (N x K uint8), alpha, zero (N fp32)."""
     _check(_quantize(_ptr(w), dtype, N, K, _ptr(q), _ptr(alpha), _ptr(zero), _stream(stream)))
+
+
+def quantize_int8_clipped(w, dtype: int, N: int, K: int, gamma, beta, q, alpha, zero,
+                          stream=None) -> None:
+    """Eq. 3: OmniQuant-clipped container with per-row gamma, beta (N fp32)."""
+    _check(_quantize_clipped(_ptr(w), dtype, N, K, _ptr(gamma), _ptr(beta), _ptr(q), _ptr(alpha),
+                             _ptr(zero), _stream(stream)))
 
 
 def slice_pack(q, N: int, K: int, r: int, packed, stream=None) -> None:
@@ -173,4 +183,5 @@ def raw_status(fn_name: str, *args) -> int:
     """Calls a C entry point and returns its status code without raising
     (used by tests of the argument checks)."""
     return {"mq_quantize_int8": _quantize, "mq_slice_pack": _slice_pack,
+            "mq_quantize_int8_clipped": _quantize_clipped,
             "mq_linear": _linear, "mq_linear_noalloc": _linear_noalloc}[fn_name](*args)

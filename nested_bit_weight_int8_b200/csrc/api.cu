@@ -126,8 +126,26 @@ mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K, uint8
   if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return fail(MQ_ERR_UNSUPPORTED, "mq_quantize_int8: N or K too large");
   if (!aligned(w, 4) || !aligned(alpha, 4) || !aligned(zero, 4))
     return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: w, alpha, zero must be 4-byte aligned");
-  cudaError_t e = launch_quantize(w, dtype, N, K, q, alpha, zero, static_cast<cudaStream_t>(stream), sm_count());
+  cudaError_t e = launch_quantize(w, dtype, N, K, nullptr, nullptr, q, alpha, zero,
+                                  static_cast<cudaStream_t>(stream), sm_count());
   if (e != cudaSuccess) return cuda_fail(e, "mq_quantize_int8");
+  return MQ_OK;
+}
+
+mq_status mq_quantize_int8_clipped(const void* w, int dtype, int64_t N, int64_t K,
+                                   const float* gamma, const float* beta, uint8_t* q, float* alpha,
+                                   float* zero, void* stream) {
+  g_last_error.clear();
+  if (!w || !gamma || !beta || !q || !alpha || !zero)
+    return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8_clipped: null pointer");
+  if (dtype != MQ_F32 && dtype != MQ_BF16) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8_clipped: dtype must be MQ_F32 or MQ_BF16");
+  if (N < 1 || K < 1) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8_clipped: N and K must be >= 1");
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return fail(MQ_ERR_UNSUPPORTED, "mq_quantize_int8_clipped: N or K too large");
+  if (!aligned(w, 4) || !aligned(alpha, 4) || !aligned(zero, 4) || !aligned(gamma, 4) || !aligned(beta, 4))
+    return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8_clipped: w, gamma, beta, alpha, zero must be 4-byte aligned");
+  cudaError_t e = launch_quantize(w, dtype, N, K, gamma, beta, q, alpha, zero,
+                                  static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "mq_quantize_int8_clipped");
   return MQ_OK;
 }
 

@@ -57,8 +57,10 @@ cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uin
                           bool swizzle128 = false);
 int sm_count();
 
-cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
-                            float* alpha, float* zero, cudaStream_t stream, int sms);
+// gamma, beta: per-row clipping factors of Eq. 3, or null for Eq. 1.
+cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, const float* gamma,
+                            const float* beta, uint8_t* q, float* alpha, float* zero,
+                            cudaStream_t stream, int sms);
 cudaError_t launch_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* packed,
                               cudaStream_t stream, int sms);
 

@@ -51,10 +51,13 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
 // One CTA per row (grid-stride over rows). Pass 1 reduces min and max; one
 // thread derives alpha and z; pass 2 re-reads the row (an L2 hit) and writes
 // the codes. `vec` selects 8-element vector accesses (K % 16 == 0 and every
-// pointer 16-byte aligned), else element accesses.
+// pointer 16-byte aligned), else element accesses. With `gamma` and `beta`
+// (one pair per row) the range is OmniQuant's clipped [beta*min, gamma*max]
+// (Eq. 3) and weights outside it saturate; without them it is Eq. 1's.
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_rows_kernel(const T* __restrict__ w, int64_t N, int64_t K, bool vec,
+                     const float* __restrict__ gamma, const float* __restrict__ beta,
                      uint8_t* __restrict__ q, float* __restrict__ alpha,
                      float* __restrict__ zero) {
   __shared__ float s_mn[kQuantThreads / 32], s_mx[kQuantThreads / 32];
@@ -88,9 +91,14 @@ quantize_rows_kernel(const T* __restrict__ w, int64_t N, int64_t K, bool vec,
     if (tid == 0) {
       float a = s_mn[0], b = s_mx[0];
       for (int i = 1; i < kQuantThreads / 32; ++i) { a = fminf(a, s_mn[i]); b = fmaxf(b, s_mx[i]); }
+      if (gamma) {  // Eq. 3: the clipped range [beta * min, gamma * max]
+        b = __fmul_rn(gamma[n], b);
+        a = __fmul_rn(beta[n], a);
+      }
       // Eq. 1: alpha = (max - min) / (2^8 - 1), z = -min / alpha.
       float al = __fdiv_rn(__fsub_rn(b, a), 255.0f);
-      if (al == 0.0f) al = 1.0f;   // constant row: every code 0, alpha*(0 - z) = min
+      // constant row (or an empty clipped range): alpha = 1, z = -min
+      if (!(al > 0.0f)) al = 1.0f;
       const float z = __fdiv_rn(-a, al);
       s_alpha = al;
       s_zero = z;
@@ -207,18 +215,19 @@ int grid_for(int64_t work, int threads, int sms) {
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
-                            float* alpha, float* zero, cudaStream_t stream, int sms) {
+cudaError_t launch_quantize(const void* w, int dtype, int64_t N, int64_t K, const float* gamma,
+                            const float* beta, uint8_t* q, float* alpha, float* zero,
+                            cudaStream_t stream, int sms) {
   const bool aligned = ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(q)) & 15) == 0;
   const bool vec = aligned && (K % 16 == 0);
   int64_t grid = N < int64_t(sms) * 8 ? N : int64_t(sms) * 8;
   if (grid < 1) grid = 1;
   if (dtype == 0) {
     quantize_rows_kernel<float><<<static_cast<int>(grid), kQuantThreads, 0, stream>>>(
-        static_cast<const float*>(w), N, K, vec, q, alpha, zero);
+        static_cast<const float*>(w), N, K, vec, gamma, beta, q, alpha, zero);
   } else {
     quantize_rows_kernel<__nv_bfloat16><<<static_cast<int>(grid), kQuantThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(w), N, K, vec, q, alpha, zero);
+        static_cast<const __nv_bfloat16*>(w), N, K, vec, gamma, beta, q, alpha, zero);
   }
   return cudaGetLastError();
 }

@@ -65,6 +65,13 @@ def student_t_weights(n: int, k: int, seed: int, nu: float = 4.0, scale: float =
     return w if dtype == "f32" else bf16_bits_from_f32(w)
 
 
+def clip_factors(n: int, seed: int, lo: float = 0.6, hi: float = 1.0) -> np.ndarray:
+    """Per-row clipping factors for Eq. 3 (gamma or beta): uniform in [lo, hi],
+    float32. OmniQuant learns them through a sigmoid, so they lie in (0, 1);
+    no training runs here, so they are drawn."""
+    return _rng(seed).uniform(lo, hi, size=n).astype(np.float32)
+
+
 def activations(m: int, k: int, seed: int) -> np.ndarray:
     """bf16 activations x ~ N(0, 1), m rows by k features, as uint16 bits."""
     x = _rng(seed).standard_normal((m, k), dtype=np.float64).astype(np.float32)
