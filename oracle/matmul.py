@@ -21,9 +21,10 @@ from .slicing import slice_codes
 
 
 def dequant_slice(q: np.ndarray, alpha: np.ndarray, zero: np.ndarray, r: int,
-                  c: int = 8) -> np.ndarray:
-    """W_r = alpha * (S(q, r) - z) in float64, N x K."""
-    s_val = slice_codes(q, r, c).astype(np.float64) * float(1 << (c - r))
+                  c: int = 8, clamp: bool = True) -> np.ndarray:
+    """W_r = alpha * (S(q, r) - z) in float64, N x K (S from Eq. 6, or from
+    the unclamped Eq. 8 when clamp=False)."""
+    s_val = slice_codes(q, r, c, clamp).astype(np.float64) * float(1 << (c - r))
     a = np.asarray(alpha, dtype=np.float64)[:, None]
     z = np.asarray(zero, dtype=np.float64)[:, None]
     return a * (s_val - z)

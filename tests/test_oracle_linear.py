@@ -112,3 +112,35 @@ def test_pins_catch_transposed_matmul():
     xs = np.random.default_rng(3).standard_normal((1, 32))
     assert not np.allclose(oracle.linear(xs, sq), xs @ sq)
     assert oracle.linear(x, wr).shape == (2, 3)
+
+
+def test_unclamped_dequant_int2_value_set():
+    # Eq. 8 (no clamp) at r = 2 over every container value, alpha = 1, z = 0:
+    # the errata paragraph's five levels {0, 64, 128, 192, 256}; the top one
+    # is reached exactly from q = 224 (= 256 - 2^(s-1)) upward, and below it
+    # the two forms agree
+    q = np.arange(256, dtype=np.uint8)[None, :]
+    one, zero = np.ones(1, np.float32), np.zeros(1, np.float32)
+    ep = oracle.dequant_slice(q, one, zero, 2, clamp=False)[0]
+    cl = oracle.dequant_slice(q, one, zero, 2)[0]
+    assert set(ep.tolist()) == {0.0, 64.0, 128.0, 192.0, 256.0}
+    assert np.array_equal(np.nonzero(ep == 256.0)[0], np.arange(224, 256))
+    assert np.array_equal(ep[:224], cl[:224]) and np.all(cl[224:] == 192.0)
+
+
+@pytest.mark.parametrize("r", [6, 4, 3, 2])
+def test_unclamped_exact_rational_brute_force(r):
+    # y with Eq. 8's unclamped codes, summed in exact rationals; each row's
+    # maximum quantizes to q = 255, which lands in the extra bucket 2^r
+    w, x = _small(seed=4)
+    q, a, z = oracle.quantize_minmax(w)
+    assert (q == 255).any(axis=1).all()
+    y = oracle.linear(x, oracle.dequant_slice(q, a, z, r, clamp=False))
+    s = 8 - r
+    for m in range(x.shape[0]):
+        for n in range(w.shape[0]):
+            acc = Fraction(0)
+            for kk in range(w.shape[1]):
+                code = (int(q[n, kk]) + 2 ** (s - 1)) >> s  # round half up, no clamp
+                acc += Fraction(x[m, kk]) * Fraction(float(a[n])) * (code * 2 ** s - Fraction(float(z[n])))
+            assert abs(float(acc) - y[m, n]) <= 1e-12 * (1 + abs(float(acc)))
