@@ -240,8 +240,10 @@ def time_device(fn, steps: int, warmup: int, stream, world: int, dev):
 
 def rows_timings(dev, stream):
     """Separately timed rows of the path on one 14336x4096 bf16 weight:
-    quantize (Eq. 1 and Eq. 3's clipped variant), slice-pack (Eq. 6) per width, one decode linear per
-    width (M = 1), and the prefill GEMM at M = 2048 when served."""
+    quantize (Eq. 1 and Eq. 3's clipped variant), slice-pack (Eq. 6) per
+    width, one decode linear per width (M = 1), the decode linear sliced on
+    load from the container (Eq. 6 and Eq. 8), Extra Precision from the r = 2
+    planes plus its sparse list, and the prefill GEMM at M = 2048."""
     import torch
     import nested_bit_weight_int8_b200 as mq
     n, k = 14336, 4096
@@ -291,6 +293,39 @@ def rows_timings(dev, stream):
         out[f"slice_pack_r{r}"] = {"us": round(us, 2), "GBps": round((n * k + n * k * r // 8) / us / 1e3, 1)}
         us = timed(lambda: mq.linear(x, 1, k, p, a, z, n, r, y, stream))
         out[f"decode_linear_r{r}_M1"] = {"us": round(us, 2), "GBps": round(n * k * r / 8 / us / 1e3, 1)}
+    # Extra Precision (Eq. 8) from the r = 2 planes plus the sparse list of
+    # extra-bucket positions, on weights with about 2.5% of each row there
+    we = torch.randn((n, k), generator=gen, device=dev).clamp_(-4.0, 4.0)
+    top = torch.rand((n, k), generator=gen, device=dev) < 0.025
+    we = torch.where(top, 3.2 + 0.8 * torch.rand((n, k), generator=gen, device=dev), we)
+    we[:, 0] = -4.0
+    we[:, 1] = 4.0
+    we = (we * 0.02).to(torch.bfloat16)
+    qe = torch.empty_like(q)
+    ae, ze = torch.empty_like(a), torch.empty_like(z)
+    mq.quantize_int8(we, mq.MQ_BF16, n, k, qe, ae, ze, stream)
+    del we, top
+    pe = torch.empty(mq.packed_bytes(n, k, 2), dtype=torch.uint8, device=dev)
+    mq.slice_pack(qe, n, k, 2, pe, stream)
+    rows_e = torch.empty(n + 1, dtype=torch.int32, device=dev)
+    mq.ep_overflow_rows(qe, n, k, 2, rows_e, stream)
+    torch.cuda.synchronize()
+    nnz = int(rows_e[n].item())
+    cols_e = torch.empty(max(nnz, 8), dtype=torch.int16, device=dev)
+    mq.ep_overflow_cols(qe, n, k, 2, rows_e, cols_e, stream)
+    us = timed(lambda: mq.linear_ep(x, 1, k, pe, ae, ze, n, 2, rows_e, cols_e, y, stream))
+    ep_bytes = n * k * 2 // 8 + 2 * nnz + 4 * (n + 1)
+    out["decode_linear_ep_r2_M1"] = {"us": round(us, 2), "GBps": round(ep_bytes / us / 1e3, 1),
+                                     "extra_bucket_frac": round(nnz / (n * k), 4),
+                                     "bits_per_weight": round(8 * ep_bytes / (n * k), 3)}
+    us = timed(lambda: mq.linear(x, 1, k, pe, ae, ze, n, 2, y, stream))
+    out["decode_linear_eq6_same_planes_r2_M1"] = {"us": round(us, 2)}
+    del qe, pe, rows_e, cols_e
+    # slice on load from the int8 container (8 bits per weight streamed)
+    for r in (4, 2):
+        for clamp, tag in ((True, "eq6"), (False, "eq8")):
+            us = timed(lambda: mq.linear_container(x, 1, k, q, a, z, n, r, clamp, y, stream))
+            out[f"decode_container_r{r}_{tag}_M1"] = {"us": round(us, 2), "GBps": round(n * k / us / 1e3, 1)}
     # prefill GEMM on the 9B-shaped matrices, M = 2048, the interpolative widths
     bf16_peak = _peaks()[1]
     m = 2048

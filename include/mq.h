@@ -142,6 +142,60 @@ MQ_API mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* pack
                     const float* alpha, const float* zero, int64_t N, int r,
                     float* y, void* stream);
 
+/*
+ * Slice on load: the product of mq_linear served straight from the int8
+ * container, with no repacked planes (the pages' "extracted on the fly by
+ * slicing"). Each byte is sliced as the weights stream, s = 8 - r:
+ *   clamp = 1, Eq. 6:  code = min(round_half_up(q / 2^s), 2^r - 1);
+ *   clamp = 0, Eq. 8 (the Extra Precision variant of the errata section):
+ *                      code = round_half_up(q / 2^s), which reaches 2^r for
+ *                      q >= 256 - 2^(s-1), so 2^r + 1 levels;
+ *   y[m,n] = sum_k x[m,k] * alpha_n * (code[n,k] * 2^s - z_n).
+ * It streams 8 bits per weight: it saves the planes' storage, not bandwidth.
+ *   q : N x K uint8 container (row pitch K bytes), 16-byte aligned.
+ *   Other arguments and the accuracy bound as mq_linear. Requires
+ *   1 <= M <= 32 (the decode path; larger M returns MQ_ERR_UNSUPPORTED),
+ *   K % 128 == 0, clamp in {0, 1}. At r = 8 both forms are the container.
+ */
+MQ_API mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t* q,
+                                     const float* alpha, const float* zero, int64_t N, int r,
+                                     int clamp, float* y, void* stream);
+
+/*
+ * Extra Precision on the planes (the errata section's Eq. 8, the clamp of
+ * Eq. 6 removed): at width r, s = 8 - r, the unclamped code of q is one step
+ * (2^s on the 8-bit scale) above the clamped one exactly for
+ * q >= 256 - 2^(s-1), the "extra bucket". Those positions are few, so they
+ * are kept as a sparse list beside the r-bit planes of Eq. 6, in compressed
+ * sparse rows: row n's columns are cols[row_ptr[n] .. row_ptr[n+1]),
+ * increasing. Build it in two calls: mq_ep_overflow_rows fills row_ptr
+ * (N + 1 int32: counts and their scan, row_ptr[0] = 0); read row_ptr[N]
+ * (the total) to size cols; mq_ep_overflow_cols fills cols (uint16).
+ *   q : N x K uint8 container, 16-byte aligned, K % 16 == 0, K <= 65536,
+ *       N * K < 2^31. r in {6, 4, 3, 2} (r = 8 has no extra bucket).
+ *   row_ptr : N + 1 int32 (device), 4-byte aligned. cols : row_ptr[N]
+ *       uint16 (device), 2-byte aligned.
+ */
+MQ_API mq_status mq_ep_overflow_rows(const uint8_t* q, int64_t N, int64_t K, int r,
+                                     int32_t* row_ptr, void* stream);
+MQ_API mq_status mq_ep_overflow_cols(const uint8_t* q, int64_t N, int64_t K, int r,
+                                     const int32_t* row_ptr, uint16_t* cols, void* stream);
+
+/*
+ * The Extra Precision product from the Eq. 6 planes plus the sparse list:
+ *   y[m,n] = sum_k x[m,k] alpha_n (code8[n,k] 2^s - z_n),
+ * code8 the unclamped Eq. 8 code, computed as the planes' product plus
+ * alpha_n 2^s sum over row n's listed positions of x[m,k] (the "sparse
+ * additions"), fused into the decode kernel's epilogue. Arguments as
+ * mq_linear plus the list of mq_ep_overflow_*; requires 1 <= M <= 32 (larger
+ * M returns MQ_ERR_UNSUPPORTED), r in {6, 4, 3, 2}, K <= 65536. Accuracy as
+ * mq_linear, against W with the Eq. 8 codes.
+ */
+MQ_API mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed,
+                              const float* alpha, const float* zero, int64_t N, int r,
+                              const int32_t* row_ptr, const uint16_t* cols, float* y,
+                              void* stream);
+
 /* One linear of a stack: its input, its packed planes, its scales, its output. */
 typedef struct mq_linear_desc {
   const void* x;       /* M x K bf16 input, 16-byte aligned */

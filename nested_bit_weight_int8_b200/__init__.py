@@ -54,6 +54,12 @@ _linear = _sig("mq_linear", _int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _
 _stack = _sig("mq_stack_forward", _int,
               [ctypes.POINTER(LinearDesc), ctypes.POINTER(_int), _int, ctypes.POINTER(_int), _int,
                _i64, _vp])
+_linear_container = _sig("mq_linear_container", _int,
+                         [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _int, _vp, _vp])
+_ovf_rows = _sig("mq_ep_overflow_rows", _int, [_vp, _i64, _i64, _int, _vp, _vp])
+_ovf_cols = _sig("mq_ep_overflow_cols", _int, [_vp, _i64, _i64, _int, _vp, _vp, _vp])
+_linear_ep = _sig("mq_linear_ep", _int,
+                  [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _vp])
 _linear_noalloc = _sig("mq_linear_noalloc", _int,
                       [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
 _device_status = _sig("mq_device_status", _int, [_vp])
@@ -63,7 +69,8 @@ _wait_limit = _sig("mq_debug_set_wait_limit_ns", _int, [_u64])
 EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8",
             "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
             "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc",
-            "mq_quantize_int8_clipped")
+            "mq_quantize_int8_clipped", "mq_linear_container", "mq_ep_overflow_rows",
+            "mq_ep_overflow_cols", "mq_linear_ep")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -130,6 +137,32 @@ def linear(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=Non
                    _stream(stream)))
 
 
+def linear_container(x, M: int, K: int, q, alpha, zero, N: int, r: int, clamp: bool, y,
+                     stream=None) -> None:
+    """Slice on load: y = x . W_r^T read straight from the int8 container q,
+    sliced by Eq. 6 (clamp=True) or the unclamped Eq. 8 (clamp=False)."""
+    _check(_linear_container(_ptr(x), M, K, _ptr(q), _ptr(alpha), _ptr(zero), N, r,
+                             1 if clamp else 0, _ptr(y), _stream(stream)))
+
+
+def ep_overflow_rows(q, N: int, K: int, r: int, row_ptr, stream=None) -> None:
+    """Extra Precision list, step 1: row_ptr (N + 1 int32) = scan of the
+    per-row counts of positions whose Eq. 8 code exceeds the Eq. 6 code."""
+    _check(_ovf_rows(_ptr(q), N, K, r, _ptr(row_ptr), _stream(stream)))
+
+
+def ep_overflow_cols(q, N: int, K: int, r: int, row_ptr, cols, stream=None) -> None:
+    """Extra Precision list, step 2: cols (row_ptr[N] uint16) = those positions."""
+    _check(_ovf_cols(_ptr(q), N, K, r, _ptr(row_ptr), _ptr(cols), _stream(stream)))
+
+
+def linear_ep(x, M: int, K: int, packed, alpha, zero, N: int, r: int, row_ptr, cols, y,
+              stream=None) -> None:
+    """Eq. 8 (Extra Precision) product: the Eq. 6 planes plus the sparse list."""
+    _check(_linear_ep(_ptr(x), M, K, _ptr(packed), _ptr(alpha), _ptr(zero), N, r, _ptr(row_ptr),
+                      _ptr(cols), _ptr(y), _stream(stream)))
+
+
 def linear_noalloc(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=None) -> None:
     """As linear() for 1 <= M <= 32, but working in the library's fixed device
     array instead of allocating a workspace (for callers that cannot allocate).
@@ -184,4 +217,6 @@ def raw_status(fn_name: str, *args) -> int:
     (used by tests of the argument checks)."""
     return {"mq_quantize_int8": _quantize, "mq_slice_pack": _slice_pack,
             "mq_quantize_int8_clipped": _quantize_clipped,
-            "mq_linear": _linear, "mq_linear_noalloc": _linear_noalloc}[fn_name](*args)
+            "mq_linear": _linear, "mq_linear_noalloc": _linear_noalloc,
+            "mq_linear_container": _linear_container, "mq_linear_ep": _linear_ep,
+            "mq_ep_overflow_rows": _ovf_rows, "mq_ep_overflow_cols": _ovf_cols}[fn_name](*args)

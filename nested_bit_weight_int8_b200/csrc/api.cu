@@ -193,6 +193,69 @@ mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed, con
   return MQ_OK;
 }
 
+mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t* q,
+                              const float* alpha, const float* zero, int64_t N, int r, int clamp,
+                              float* y, void* stream) {
+  g_last_error.clear();
+  mq_status st = check_linear("mq_linear_container", x, M, K, q, alpha, zero, N, r, y);
+  if (st != MQ_OK) return st;
+  if (clamp != 0 && clamp != 1) return fail(MQ_ERR_INVALID_ARG, "mq_linear_container: clamp must be 0 or 1");
+  if (M > 32) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_container: M must be <= 32 (decode path)");
+  LinearJob job{x, q, alpha, zero, y, N, K, r, clamp ? kContainer : kContainerEP};
+  cudaError_t e = run_gemv(&job, 1, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mq_linear_container");
+  return MQ_OK;
+}
+
+static mq_status check_ovf(const char* who, const uint8_t* q, int64_t N, int64_t K, int r) {
+  if (!q) return fail(MQ_ERR_INVALID_ARG, "%s: null q", who);
+  if (r != 6 && r != 4 && r != 3 && r != 2) return fail(MQ_ERR_INVALID_ARG, "%s: r=%d not in {6,4,3,2}", who, r);
+  if (N < 1 || K < 16 || K % 16 != 0) return fail(MQ_ERR_INVALID_ARG, "%s: need N >= 1 and K a positive multiple of 16", who);
+  if (K > 65536 || N * K >= (int64_t(1) << 31)) return fail(MQ_ERR_UNSUPPORTED, "%s: K > 65536 or N*K >= 2^31", who);
+  if (!aligned(q, 16)) return fail(MQ_ERR_INVALID_ARG, "%s: q must be 16-byte aligned", who);
+  return MQ_OK;
+}
+
+mq_status mq_ep_overflow_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32_t* row_ptr,
+                              void* stream) {
+  g_last_error.clear();
+  mq_status st = check_ovf("mq_ep_overflow_rows", q, N, K, r);
+  if (st != MQ_OK) return st;
+  if (!row_ptr || !aligned(row_ptr, 4)) return fail(MQ_ERR_INVALID_ARG, "mq_ep_overflow_rows: row_ptr null or not 4-byte aligned");
+  cudaError_t e = launch_ovf_rows(q, N, K, r, row_ptr, static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "mq_ep_overflow_rows");
+  return MQ_OK;
+}
+
+mq_status mq_ep_overflow_cols(const uint8_t* q, int64_t N, int64_t K, int r, const int32_t* row_ptr,
+                              uint16_t* cols, void* stream) {
+  g_last_error.clear();
+  mq_status st = check_ovf("mq_ep_overflow_cols", q, N, K, r);
+  if (st != MQ_OK) return st;
+  if (!row_ptr || !aligned(row_ptr, 4)) return fail(MQ_ERR_INVALID_ARG, "mq_ep_overflow_cols: row_ptr null or not 4-byte aligned");
+  if (!cols || !aligned(cols, 2)) return fail(MQ_ERR_INVALID_ARG, "mq_ep_overflow_cols: cols null or not 2-byte aligned");
+  cudaError_t e = launch_ovf_cols(q, N, K, r, row_ptr, cols, static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "mq_ep_overflow_cols");
+  return MQ_OK;
+}
+
+mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed, const float* alpha,
+                       const float* zero, int64_t N, int r, const int32_t* row_ptr,
+                       const uint16_t* cols, float* y, void* stream) {
+  g_last_error.clear();
+  mq_status st = check_linear("mq_linear_ep", x, M, K, packed, alpha, zero, N, r, y);
+  if (st != MQ_OK) return st;
+  if (r == 8) return fail(MQ_ERR_INVALID_ARG, "mq_linear_ep: r=8 has no extra bucket");
+  if (!row_ptr || !cols || !aligned(row_ptr, 4) || !aligned(cols, 2))
+    return fail(MQ_ERR_INVALID_ARG, "mq_linear_ep: row_ptr / cols null or misaligned");
+  if (K > 65536) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: K > 65536");
+  if (M > 32) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: M must be <= 32 (decode path)");
+  LinearJob job{x, static_cast<const uint8_t*>(packed), alpha, zero, y, N, K, r, kPlanes, row_ptr, cols};
+  cudaError_t e = run_gemv(&job, 1, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mq_linear_ep");
+  return MQ_OK;
+}
+
 mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, int n_lins,
                            const int* widths, int n_layers, int64_t M, void* stream) {
   g_last_error.clear();

@@ -30,6 +30,15 @@
 //   y = A_n (acc - O_m) - B_n Sx_m,  A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n.
 // Offsets stay <= 384, so fp32 partial sums stay small (accuracy), and
 // two codes are decoded per shift+LOP3 pair (issue budget at r = 2).
+//
+// Slicing on load. A linear may also stream the int8 container itself (the
+// r = 8 plane) and slice each byte while decoding, so one stored matrix serves
+// every width with no repack ("extracted on the fly by slicing"): the code is
+// (q + 2^(s-1)) >> s, s = 8 - r, clamped to 2^r - 1 by Eq. 6 or left at up to
+// 2^r by the unclamped Eq. 8 (the Extra Precision variant). Two bytes sit in
+// the 16-bit halves of a register; the rounding add (and Eq. 6's clamp) runs
+// on both halves at once, and a shift and a LOP3 place the code under a bf16
+// power of two, as for the planes.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -85,6 +94,13 @@ struct LinDesc {
   const uint8_t* xf;   // activations in fragment order, n_kc blocks of M*KC bf16
   const float* psum;   // [M][8] activation sums per class (k >> 1) & 7
   int N, K, r, kc, n_kc, unit_begin;
+  int dk;  // decode kind: r for planes, 10 / 11 for the container sliced by Eq. 6 / Eq. 8
+  // Extra Precision on the planes (or null): row n's positions whose Eq. 8
+  // code is one step above the Eq. 6 code are ep_cols[ep_rows[n] .. ep_rows[n+1]),
+  // gathered from the activations x (M x K bf16).
+  const int* ep_rows;
+  const uint16_t* ep_cols;
+  const __nv_bfloat16* x;
 };
 
 template <int CAP>
@@ -101,6 +117,8 @@ struct GemvParams {
   int cta_begin[kMaxCtas + 1];  // unit range of CTA c: [cta_begin[c], cta_begin[c + 1])
   LinDesc lin[CAP];
 };
+// kernel parameters are limited to 32764 bytes
+static_assert(sizeof(GemvParams<kGemvMaxLinears>) <= 32764, "decode kernel parameters too large");
 
 // Geometry of one width: plane widths, 8-code activation groups per 16-byte
 // low-plane chunk (W8).
@@ -110,9 +128,35 @@ template <> struct Geo<4> { static constexpr int b0 = 4, b1 = 0, W8 = 4; };
 template <> struct Geo<8> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
 template <> struct Geo<3> { static constexpr int b0 = 2, b1 = 1, W8 = 8; };
 template <> struct Geo<6> { static constexpr int b0 = 4, b1 = 2, W8 = 4; };
+// The container sliced on load (Eq. 6: kind 10, Eq. 8: kind 11) streams the
+// 8-bit plane.
+template <> struct Geo<10> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
+template <> struct Geo<11> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
+
+// Per-linear constants of the slice-on-load decode (both 16-bit halves):
+// h2 the rounding addend 2^(s-1), kmask the code's bits after the shift, mag
+// the bf16 power of two the code is OR-ed under (code weight 1).
+struct Cdec {
+  uint32_t h2, kmask, mag;
+};
+__device__ __forceinline__ Cdec make_cdec(int dk, int r) {
+  Cdec c{0u, 0u, 0u};
+  if (dk == 10 || dk == 11) {
+    const int s = 8 - r;
+    c.h2 = (1u << (s - 1)) * 0x10001u;
+    // Eq. 6: min(q + h, 255) >> 1 holds the r-bit code at bits 7-r .. 6, under
+    // 2^r. Eq. 8: (q + h) >> 2 holds the (r+1)-bit code at bits 6-r .. 6,
+    // under 2^(r+1).
+    const int e = dk == 10 ? r : r + 1;
+    const uint32_t bits = dk == 10 ? ((1u << r) - 1u) << (7 - r) : ((1u << (r + 1)) - 1u) << (6 - r);
+    c.kmask = bits * 0x10001u;
+    c.mag = (static_cast<uint32_t>(127 + e) << 7) * 0x10001u;
+  }
+  return c;
+}
 
 __device__ __forceinline__ void plane_widths_dev(int r, int& b0, int& b1) {
-  b0 = (r == 8) ? 8 : (r == 4 || r == 6) ? 4 : 2;
+  b0 = (r == 8 || r >= 10) ? 8 : (r == 4 || r == 6) ? 4 : 2;  // 10, 11: the container
   b1 = (r == 3) ? 1 : (r == 6) ? 2 : 0;
 }
 
@@ -169,8 +213,21 @@ __device__ __forceinline__ uint32_t pick2(uint32_t w) {
 // plane; Q is the 8-code group of the chunk, HF the 4-code half of it.
 template <int R, int PLANE, int Q, int HF>
 __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint32_t (&hi)[2],
-                                            uint32_t& x0, uint32_t& x1) {
-  if constexpr (R == 2) {
+                                            const Cdec& cd, uint32_t& x0, uint32_t& x1) {
+  if constexpr (R == 10 || R == 11) {
+    // container bytes c0..c3 of one word, registers pair (c0, c2) and (c1, c3)
+    // as the r = 8 plane does; q + h never leaves its 16-bit half
+    const uint32_t w = lo[2 * Q + HF];
+    const uint32_t ev = w & 0x00FF00FFu;
+    const uint32_t od = __byte_perm(w, 0u, 0x4341);
+    if constexpr (R == 10) {
+      x0 = and_or(__viaddmin_u16x2(ev, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag);
+      x1 = and_or(__viaddmin_u16x2(od, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag);
+    } else {
+      x0 = and_or((ev + cd.h2) >> 2, cd.kmask, cd.mag);
+      x1 = and_or((od + cd.h2) >> 2, cd.kmask, cd.mag);
+    }
+  } else if constexpr (R == 2) {
     // 2-bit codes, word = 16 codes; x0 holds codes 4j, 4j+1 (half-word
     // position 4j), x1 codes 4j+2, 4j+3 (position 4j+2), j = 2(Q%2)+HF.
     constexpr int j = 2 * (Q % 2) + HF;
@@ -220,13 +277,15 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
 // width (the sum over the planes of the magic added to the code). The offsets
 // stay small next to the code unit (at most 32 at r = 2), so the fp32 sums
 // lose little to cancellation when the offsets are taken out again.
-__device__ __forceinline__ void offset_coeffs(int r, float (&c)[kClasses]) {
+__device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses]) {
   constexpr float r2[kClasses] = {0.f, 32.f, 8.f, 0.f, 32.f, 8.f, 0.f, 32.f};
   constexpr float r3[4] = {80.f, 36.f, 32.f, 12.f};
   constexpr float r6[4] = {272.f, 80.f, 272.f, 80.f};
+  // the container sliced on load: one magic for every class
+  const float cont = static_cast<float>(1 << (dk == 10 ? r : r + 1));
 #pragma unroll
   for (int i = 0; i < kClasses; ++i) {
-    c[i] = r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
+    c[i] = dk >= 10 ? cont : r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
   }
 }
 
@@ -235,7 +294,7 @@ __device__ __forceinline__ void offset_coeffs(int r, float (&c)[kClasses]) {
 template <int R, int NT, int TW, int Q>
 __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, float (&ch)[TW][NT][2][4]) {
+                                           int gbase, const Cdec& cd, float (&ch)[TW][NT][2][4]) {
   uint4 xb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -255,10 +314,10 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
 #pragma unroll
       for (int T = 0; T < TW; ++T) {
         uint32_t a0, a1, a2, a3;
-        if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 0, Q, 0>(lo[T][1], hi[T][1], a1, a3); }
-        if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 1, Q, 0>(lo[T][1], hi[T][1], a1, a3); }
-        if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 0, Q, 1>(lo[T][1], hi[T][1], a1, a3); }
-        if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[T][0], hi[T][0], a0, a2); decode_quad<R, 1, Q, 1>(lo[T][1], hi[T][1], a1, a3); }
+        if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 0, Q, 0>(lo[T][1], hi[T][1], cd, a1, a3); }
+        if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 1, Q, 0>(lo[T][1], hi[T][1], cd, a1, a3); }
+        if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 0, Q, 1>(lo[T][1], hi[T][1], cd, a1, a3); }
+        if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 1, Q, 1>(lo[T][1], hi[T][1], cd, a1, a3); }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const uint32_t b0 = hf ? xb[nt].z : xb[nt].x;
@@ -273,9 +332,9 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
 template <int R, int NT, int TW, int... Qs>
 __device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, float (&ch)[TW][NT][2][4],
+                                           int gbase, const Cdec& cd, float (&ch)[TW][NT][2][4],
                                            std::integer_sequence<int, Qs...>) {
-  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, ch), ...);
+  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, cd, ch), ...);
 }
 
 // One staged unit for this warp's 16-row tiles. All sub-steps are unrolled
@@ -289,7 +348,7 @@ template <int R, int NT>
 __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* st1,
                                              const uint32_t (&xaddr)[NT],
                                              const uint32_t (&xstep)[NT], int warp, int lane,
-                                             float (&ch)[Tiling<NT>::TW][NT][2][4]) {
+                                             const Cdec& cd, float (&ch)[Tiling<NT>::TW][NT][2][4]) {
   using G = Geo<R>;
   using TL = Tiling<NT>;
   constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0, P1 = TL::P0 / 2;
@@ -318,7 +377,7 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
   }
 #pragma unroll
   for (int s = 0; s < NSUB; ++s)
-    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, ch,
+    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, cd, ch,
                           std::make_integer_sequence<int, G::W8>{});
 }
 
@@ -326,6 +385,7 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
 struct Cursor {
   int l, rb, kc;          // linear, row block, k-chunk of the current unit
   int nrb, n_kc, r, N;    // of linear l
+  int dk;                 // its decode kind (width, or 10 / 11 for the container)
 };
 
 template <int RPU, int CAP>
@@ -335,6 +395,7 @@ __device__ __forceinline__ void cursor_load(const GemvParams<CAP>& p, Cursor& c)
   c.nrb = (L.N + RPU - 1) / RPU;
   c.r = L.r;
   c.N = L.N;
+  c.dk = L.dk;
 }
 
 template <int RPU, int CAP>
@@ -360,6 +421,42 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
   }
 }
 
+// Sum of x[m, k] over the Extra Precision positions k of row n, for the batch
+// rows m this lane owns (m = 8 nt + 2t + e). With at most two batch rows the
+// four lanes that share a weight row split its positions and add their parts
+// with shuffles; otherwise each lane walks the row's list for its own batch
+// rows. Every lane of the warp calls this (the shuffles); `valid` is false for
+// rows past N.
+template <int NT>
+__device__ __forceinline__ void ep_sums(const LinDesc& L, int M, int n, bool valid, int t,
+                                        float (&s)[NT][2]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) { s[nt][0] = 0.f; s[nt][1] = 0.f; }
+  const int beg = valid ? L.ep_rows[n] : 0;
+  const int end = valid ? L.ep_rows[n + 1] : 0;
+  const bool split = M <= 2;
+  const int step = split ? 4 : 1;
+  const __nv_bfloat16* xr = L.x;
+#pragma unroll 4
+  for (int j = beg + (split ? t : 0); j < end; j += step) {
+    const int k = L.ep_cols[j];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int m = split ? e : nt * 8 + 2 * t + e;
+        if (m < M) s[nt][e] += __bfloat162float(xr[static_cast<int64_t>(m) * L.K + k]);
+      }
+  }
+  if (split) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      s[0][e] += __shfl_xor_sync(0xffffffffu, s[0][e], 1);
+      s[0][e] += __shfl_xor_sync(0xffffffffu, s[0][e], 2);
+    }
+  }
+}
+
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
 // removes the decoding offsets and the zero point (once per row, by the part
 // that starts at k-chunk 0) and writes y. A row block this CTA owns whole is
@@ -372,10 +469,14 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
   float c[kClasses];
-  offset_coeffs(L.r, c);
+  offset_coeffs(L.dk, L.r, c);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h;
+    // Extra Precision: each listed position adds one code step, A * x[m, k]
+    float es[NT][2];
+    const bool ep = kc0 == 0 && L.ep_rows != nullptr;  // uniform over the warp
+    if (ep) ep_sums<NT>(L, p.M, n, n < L.N, t, es);
     if (n >= L.N) continue;
     const float a = L.alpha[n], z = L.zero[n];
     const float A = a * scale, B = a * z;
@@ -386,6 +487,7 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
         const int m = nt * 8 + 2 * t + e;
         if (m >= p.M) continue;
         float v = tot[nt][2 * h + e];
+        if (ep) v += (p.M <= 2 ? es[0][e] : es[nt][e]);
         if (kc0 == 0) {
           const float* P = L.psum + m * kClasses;
           float O = 0.f, Sx = 0.f;
@@ -416,7 +518,7 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
                                             volatile int* s_abort, int seg, int& s, uint32_t& ph,
                                             bool active, const uint32_t (&xaddr)[NT],
                                             const uint32_t (&xstep)[NT], int warp, int lane,
-                                            float (&tot)[Tiling<NT>::TW][NT][4]) {
+                                            const Cdec& cd, float (&tot)[Tiling<NT>::TW][NT][4]) {
   constexpr int TW = Tiling<NT>::TW;
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
@@ -438,7 +540,7 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
 #pragma unroll
           for (int j = 0; j < 4; ++j) { ch[T][b][0][j] = 0.f; ch[T][b][1][j] = 0.f; }
       // the plane pitches and rows follow from the batch tiles (Tiling)
-      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, ch);
+      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, cd, ch);
 #pragma unroll
       for (int T = 0; T < TW; ++T)
 #pragma unroll
@@ -497,7 +599,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       Cursor pre_c = c;
       auto issue_weights = [&](const Cursor& cc, int s) {
         int b0, b1;
-        plane_widths_dev(cc.r, b0, b1);
+        plane_widths_dev(cc.dk, b0, b1);
         uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
         const CUtensorMap* tm = p.map_table ? p.map_table + 2 * cc.l : &p.maps[2 * cc.l];
         const uint32_t box = TL::RPU * (p.pitch0 + (b1 ? p.pitch1 : 0));
@@ -580,12 +682,15 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[T][b][i] = 0.f;
     bool ok;
-    switch (c.r) {
-      case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
-      default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, tot); break;
+    const Cdec cd = make_cdec(c.dk, c.r);
+    switch (c.dk) {
+      case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
     }
     if (!ok) break;  // outputs are undefined after a give-up; the flag says so
     if (active) {
@@ -774,7 +879,7 @@ std::map<std::pair<int, std::vector<uint64_t>>, CUtensorMap*> g_map_tables;
 
 cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
   int b0, b1;
-  plane_widths(j.r, b0, b1);
+  job_planes(j, b0, b1);
   // 128-byte plane-0 rows go with 256-row units and the 128-byte swizzle
   const uint32_t rows = P0 == 128 ? 256u : 128u;
   cudaError_t e = encode_map_2d(&out2[0], j.packed, uint64_t(j.N), uint64_t(j.K) * b0 / 8,
@@ -795,7 +900,7 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
     key.push_back(reinterpret_cast<uint64_t>(jobs[i].packed));
     key.push_back(uint64_t(jobs[i].N));
     key.push_back(uint64_t(jobs[i].K));
-    key.push_back(uint64_t(jobs[i].r));
+    key.push_back(uint64_t(jobs[i].r) | (uint64_t(jobs[i].src) << 8));
   }
   std::lock_guard<std::mutex> lk(g_cache_mutex);
   auto k2 = std::make_pair(dev, std::move(key));
@@ -825,12 +930,13 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
 // decode and MMA work grows with the codes in it: measured per-unit times of
 // single-width stacks on B200 at M = 1 put r = 2 at about 1.6x and r = 4 at
 // about 1.1x an r = 8 unit; r = 3 and 6 are estimated from their planes.
-int64_t unit_cost(int r) {
-  switch (r) {
+int64_t unit_cost(const LinearJob& j) {
+  switch (decode_kind(j)) {
     case 8: return 100;
     case 4: return 108;
     case 2: return 157;
     case 6: return 170;
+    case 10: case 11: return 110;  // one 8-bit plane, one MMA per 16 codes, more decode work
     default: return 280;  // 3
   }
 }
@@ -861,7 +967,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   for (int i = 0; i < n_jobs; ++i) {
     const LinearJob& j = jobs[i];
     int b0, b1;
-    plane_widths(j.r, b0, b1);
+    job_planes(j, b0, b1);
     if (b1) two_planes = true;
     const int kc = P0 * 8 / b0;
     const int n_kc = static_cast<int>((j.K + kc - 1) / kc);
@@ -887,6 +993,10 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     d.N = static_cast<int>(j.N);
     d.K = static_cast<int>(j.K);
     d.r = j.r;
+    d.dk = decode_kind(j);
+    d.ep_rows = j.ep_rows;
+    d.ep_cols = j.ep_cols;
+    d.x = static_cast<const __nv_bfloat16*>(j.x);
     d.kc = kc;
     d.n_kc = n_kc;
     d.unit_begin = units;
@@ -944,7 +1054,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   int64_t total_cost = 0;
   for (int i = 0; i < n_jobs; ++i) {
     const int64_t lin_units = (i + 1 < n_jobs ? gp.lin[i + 1].unit_begin : units) - gp.lin[i].unit_begin;
-    total_cost += lin_units * unit_cost(jobs[i].r);
+    total_cost += lin_units * unit_cost(jobs[i]);
   }
   int n_zero = 0;
   {
@@ -955,7 +1065,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
       // first unit whose preceding cost reaches the target
       while (li < n_jobs) {
         const int64_t lin_units = (li + 1 < n_jobs ? gp.lin[li + 1].unit_begin : units) - gp.lin[li].unit_begin;
-        const int64_t lin_cost = lin_units * unit_cost(jobs[li].r);
+        const int64_t lin_cost = lin_units * unit_cost(jobs[li]);
         if (target <= cost_before + lin_cost) break;
         cost_before += lin_cost;
         ++li;
@@ -964,7 +1074,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
       if (li >= n_jobs) {
         u = units;
       } else {
-        const int64_t w = unit_cost(jobs[li].r);
+        const int64_t w = unit_cost(jobs[li]);
         u = gp.lin[li].unit_begin + static_cast<int>((target - cost_before + w - 1) / w);
       }
       if (c == 0) u = 0;
@@ -1043,7 +1153,7 @@ size_t gemv_scratch_bytes(const LinearJob& job, int M) {
   // Same arithmetic as the planner in run_gemv_cap for one linear.
   const int P0 = tiling_p0(M);
   int b0, b1;
-  plane_widths(job.r, b0, b1);
+  job_planes(job, b0, b1);
   const int kc = P0 * 8 / b0;
   const int64_t n_kc = (job.K + kc - 1) / kc;
   size_t xf = size_t(n_kc) * M * kc * 2;

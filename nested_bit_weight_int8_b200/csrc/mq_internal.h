@@ -19,7 +19,17 @@ struct LinearJob {
   int64_t N;
   int64_t K;
   int r;
+  // Where the codes come from: kPlanes (packed r-bit planes of width r), or
+  // the int8 container itself, sliced on load with Eq. 6 (kContainer) or
+  // with the unclamped Eq. 8 (kContainerEP, 2^r + 1 levels).
+  int src = 0;
+  // Extra Precision on the planes (Eq. 8 from Eq. 6 planes plus a sparse
+  // list): per row n the positions ep_cols[ep_rows[n] .. ep_rows[n+1]) whose
+  // code is one step higher; null for none.
+  const int32_t* ep_rows = nullptr;
+  const uint16_t* ep_cols = nullptr;
 };
+constexpr int kPlanes = 0, kContainer = 1, kContainerEP = 2;
 
 // Plane widths of a width r: b0 (low bits) and b1 (high bits, 0 if none).
 inline void plane_widths(int r, int& b0, int& b1) {
@@ -31,6 +41,18 @@ inline void plane_widths(int r, int& b0, int& b1) {
     case 2: b0 = 2; b1 = 0; return;
     default: b0 = 0; b1 = 0; return;
   }
+}
+// Plane widths a job streams: the container is one 8-bit plane.
+inline void job_planes(const LinearJob& j, int& b0, int& b1) {
+  if (j.src != kPlanes) { b0 = 8; b1 = 0; return; }
+  plane_widths(j.r, b0, b1);
+}
+// Decode kind of a job in the decode kernel: the width r for planes (and for
+// the container at r = 8, whose bytes are the r = 8 plane), 10 for the
+// container sliced with Eq. 6, 11 for the container with Eq. 8.
+inline int decode_kind(const LinearJob& j) {
+  if (j.src == kPlanes || j.r == 8) return j.r;
+  return j.src == kContainer ? 10 : 11;
 }
 
 // Per-(device, stream) scratch owned by the library.
@@ -83,6 +105,13 @@ size_t gemv_scratch_bytes(const LinearJob& job, int M);
 // cudaErrorMemoryAllocation if the scratch is too small (nothing launched).
 cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
                            const FixedScratch& scratch);
+
+// Extra Precision positions of a container at width r (Eq. 8 vs Eq. 6):
+// row offsets (count + scan), then the columns.
+cudaError_t launch_ovf_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32_t* row_ptr,
+                            cudaStream_t stream, int sms);
+cudaError_t launch_ovf_cols(const uint8_t* q, int64_t N, int64_t K, int r, const int32_t* row_ptr,
+                            uint16_t* cols, cudaStream_t stream, int sms);
 
 // Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
 // cudaErrorNotSupported for shapes it does not serve (nothing launched).

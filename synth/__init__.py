@@ -65,6 +65,27 @@ def student_t_weights(n: int, k: int, seed: int, nu: float = 4.0, scale: float =
     return w if dtype == "f32" else bf16_bits_from_f32(w)
 
 
+def extra_bucket_weights(n: int, k: int, seed: int, frac: float = 0.025, std: float = 0.02,
+                         dtype: str = "bf16") -> np.ndarray:
+    """Weights whose int8 container puts about `frac` of each row in the
+    int2 extra bucket of Eq. 8 (q >= 224), as a trained Extra Precision model
+    does (about 2.5%, "2.05 effective bits"): a N(0, std^2) body clipped to
+    +-4 std, each row's range pinned to exactly [-4 std, 4 std], and `frac` of
+    the positions drawn uniformly from [3.2 std, 4 std] (above the int2
+    bucket edge at 224/255 of the range, about 3.03 std)."""
+    rng = _rng(seed)
+    w = np.clip(rng.standard_normal((n, k)), -4.0, 4.0)
+    top = rng.random((n, k)) < frac
+    w[top] = rng.uniform(3.2, 4.0, size=int(top.sum()))
+    cols = rng.integers(0, k, size=(n, 2))
+    cols[:, 1] = (cols[:, 0] + 1 + rng.integers(0, k - 1, size=n)) % k  # a second, distinct column
+    rows = np.arange(n)
+    w[rows, cols[:, 0]] = -4.0
+    w[rows, cols[:, 1]] = 4.0
+    w = (w * std).astype(np.float32)
+    return w if dtype == "f32" else bf16_bits_from_f32(w)
+
+
 def clip_factors(n: int, seed: int, lo: float = 0.6, hi: float = 1.0) -> np.ndarray:
     """Per-row clipping factors for Eq. 3 (gamma or beta): uniform in [lo, hi],
     float32. OmniQuant learns them through a sigmoid, so they lie in (0, 1);

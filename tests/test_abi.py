@@ -107,3 +107,33 @@ def test_stack_rejects_bad_layers():
         mq.stack_forward(lins, [0], [5], 1)        # width 5
     with pytest.raises(mq.MQError):
         mq.stack_forward(lins, [0], [4], 33)       # M > 32
+
+
+def test_linear_container_rejects():
+    F = FAKE
+    bad = [
+        ((F, 1, 256, F, F, F, 64, 5, 1, F), mq.MQ_ERR_INVALID_ARG),    # r
+        ((F, 1, 256, F, F, F, 64, 4, 2, F), mq.MQ_ERR_INVALID_ARG),    # clamp not 0/1
+        ((F, 1, 96, F, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),     # K % 128
+        ((F, 1, 256, F + 4, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),  # misaligned q
+        ((F, 1, 256, None, F, F, 64, 4, 0, F), mq.MQ_ERR_INVALID_ARG),   # null q
+        ((F, 33, 256, F, F, F, 64, 4, 1, F), mq.MQ_ERR_UNSUPPORTED),   # prefill batch
+    ]
+    for c, want in bad:
+        assert mq.raw_status("mq_linear_container", *c, None) == want, c
+        assert mq.last_error()
+
+
+def test_ep_entry_points_reject():
+    F = FAKE
+    assert mq.raw_status("mq_ep_overflow_rows", F, 4, 64, 8, F, None) == mq.MQ_ERR_INVALID_ARG  # r = 8
+    assert mq.raw_status("mq_ep_overflow_rows", F, 4, 40, 2, F, None) == mq.MQ_ERR_INVALID_ARG  # K % 16
+    assert mq.raw_status("mq_ep_overflow_rows", F + 8, 4, 64, 2, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_ep_overflow_rows", F, 4, 65552, 2, F, None) == mq.MQ_ERR_UNSUPPORTED
+    assert mq.raw_status("mq_ep_overflow_cols", F, 4, 64, 2, F, None, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_ep_overflow_cols", F, 4, 64, 2, F + 2, F, None) == mq.MQ_ERR_INVALID_ARG
+    ok = (F, 1, 256, F, F, F, 64)
+    assert mq.raw_status("mq_linear_ep", *ok, 8, F, F, F, None) == mq.MQ_ERR_INVALID_ARG   # r = 8
+    assert mq.raw_status("mq_linear_ep", *ok, 2, None, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_linear_ep", *ok, 2, F, F + 1, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_linear_ep", F, 33, 256, F, F, F, 64, 2, F, F, F, None) == mq.MQ_ERR_UNSUPPORTED
