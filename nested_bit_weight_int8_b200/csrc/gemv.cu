@@ -95,12 +95,10 @@ struct LinDesc {
   const float* psum;   // [M][8] activation sums per class (k >> 1) & 7
   int N, K, r, kc, n_kc, unit_begin;
   int dk;  // decode kind: r for planes, 10 / 11 for the container sliced by Eq. 6 / Eq. 8
-  // Extra Precision on the planes (or null): row n's positions whose Eq. 8
-  // code is one step above the Eq. 6 code are ep_cols[ep_rows[n] .. ep_rows[n+1]),
-  // gathered from the activations x (M x K bf16).
-  const int* ep_rows;
-  const uint16_t* ep_cols;
-  const __nv_bfloat16* x;
+  // Extra Precision on the planes (or null): epc[m * N + n] is the sum of
+  // x[m, k] over row n's positions whose Eq. 8 code is one step above the
+  // Eq. 6 code, computed by the prep kernel.
+  const float* epc;
 };
 
 template <int CAP>
@@ -421,42 +419,6 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
   }
 }
 
-// Sum of x[m, k] over the Extra Precision positions k of row n, for the batch
-// rows m this lane owns (m = 8 nt + 2t + e). With at most two batch rows the
-// four lanes that share a weight row split its positions and add their parts
-// with shuffles; otherwise each lane walks the row's list for its own batch
-// rows. Every lane of the warp calls this (the shuffles); `valid` is false for
-// rows past N.
-template <int NT>
-__device__ __forceinline__ void ep_sums(const LinDesc& L, int M, int n, bool valid, int t,
-                                        float (&s)[NT][2]) {
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) { s[nt][0] = 0.f; s[nt][1] = 0.f; }
-  const int beg = valid ? L.ep_rows[n] : 0;
-  const int end = valid ? L.ep_rows[n + 1] : 0;
-  const bool split = M <= 2;
-  const int step = split ? 4 : 1;
-  const __nv_bfloat16* xr = L.x;
-#pragma unroll 4
-  for (int j = beg + (split ? t : 0); j < end; j += step) {
-    const int k = L.ep_cols[j];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int m = split ? e : nt * 8 + 2 * t + e;
-        if (m < M) s[nt][e] += __bfloat162float(xr[static_cast<int64_t>(m) * L.K + k]);
-      }
-  }
-  if (split) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      s[0][e] += __shfl_xor_sync(0xffffffffu, s[0][e], 1);
-      s[0][e] += __shfl_xor_sync(0xffffffffu, s[0][e], 2);
-    }
-  }
-}
-
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
 // removes the decoding offsets and the zero point (once per row, by the part
 // that starts at k-chunk 0) and writes y. A row block this CTA owns whole is
@@ -473,10 +435,6 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h;
-    // Extra Precision: each listed position adds one code step, A * x[m, k]
-    float es[NT][2];
-    const bool ep = kc0 == 0 && L.ep_rows != nullptr;  // uniform over the warp
-    if (ep) ep_sums<NT>(L, p.M, n, n < L.N, t, es);
     if (n >= L.N) continue;
     const float a = L.alpha[n], z = L.zero[n];
     const float A = a * scale, B = a * z;
@@ -487,8 +445,9 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
         const int m = nt * 8 + 2 * t + e;
         if (m >= p.M) continue;
         float v = tot[nt][2 * h + e];
-        if (ep) v += (p.M <= 2 ? es[0][e] : es[nt][e]);
         if (kc0 == 0) {
+          // Extra Precision: each listed position adds one code step
+          if (L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
           const float* P = L.psum + m * kClasses;
           float O = 0.f, Sx = 0.f;
 #pragma unroll
@@ -727,14 +686,26 @@ struct PrepZero {
   float* y;
   int N, rb;
 };
+// Extra Precision sums of one linear: out[m * N + n] = sum over row n's
+// listed positions k (cols[rows[n] .. rows[n + 1])) of x[m, k].
+struct PrepEp {
+  const int* rows;
+  const uint16_t* cols;
+  const __nv_bfloat16* x;
+  float* out;
+  int N, K;
+};
+constexpr int kMaxEpJobs = 8;
 template <int CAP>
 struct PrepParams {
-  int M, n_layout, n_sum, n_zero;
+  int M, n_layout, n_sum, n_zero, n_ep;
   int rows;  // weight rows per unit: the height of a zeroed row block
   PrepLayout lay[CAP];
   PrepSum sum[CAP];
   PrepZero zero[kMaxCtas];
+  PrepEp ep[kMaxEpJobs];
 };
+static_assert(sizeof(PrepParams<kGemvMaxLinears>) <= 32764, "prep kernel parameters too large");
 
 // Builds the fragment-ordered activation blocks (zero-padded to whole
 // k-chunks) and the per-class activation sums, and zeroes the output row
@@ -801,6 +772,33 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       const int64_t off = int64_t(kc) * M * L.kc * 2 +
                           ((int64_t(s * L.w8 + q) * M + m) * 4 + t) * 16;
       *reinterpret_cast<uint4*>(L.xf + off) = v;
+    }
+  }
+  // (4) Extra Precision sums: one warp per (job, row). With M' the next power
+  // of two >= M, lane l takes batch row l % M' and every (32 / M')-th listed
+  // position; lanes of one batch row then add up with shuffles.
+  if (p.n_ep > 0) {
+    int mp = 1;
+    while (mp < M) mp <<= 1;
+    const int lane = threadIdx.x & 31;
+    const int m = lane & (mp - 1), jo = lane / mp, P = 32 / mp;
+    const int64_t warps = stride / 32;
+    int64_t total_rows = 0;
+    for (int i = 0; i < p.n_ep; ++i) total_rows += p.ep[i].N;
+    for (int64_t w = tid / 32; w < total_rows; w += warps) {
+      int job = 0;
+      int64_t n = w;
+      while (n >= p.ep[job].N) { n -= p.ep[job].N; ++job; }
+      const PrepEp& E = p.ep[job];
+      const int beg = E.rows[n], end = E.rows[n + 1];
+      float acc = 0.f;
+      if (m < M) {
+        const __nv_bfloat16* xr = E.x + int64_t(m) * E.K;
+#pragma unroll 4
+        for (int j = beg + jo; j < end; j += P) acc += __bfloat162float(xr[E.cols[j]]);
+      }
+      for (int o = mp; o < 32; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (jo == 0 && m < M) E.out[int64_t(m) * E.N + n] = acc;
     }
   }
   // (3) zero the shared output row blocks
@@ -994,9 +992,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     d.K = static_cast<int>(j.K);
     d.r = j.r;
     d.dk = decode_kind(j);
-    d.ep_rows = j.ep_rows;
-    d.ep_cols = j.ep_cols;
-    d.x = static_cast<const __nv_bfloat16*>(j.x);
+    d.epc = nullptr;  // set with the workspace below
     d.kc = kc;
     d.n_kc = n_kc;
     d.unit_begin = units;
@@ -1013,7 +1009,16 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     if (em != cudaSuccess) return em;
   }
   const size_t psum_off = xf_bytes;
-  const size_t ws_bytes = psum_off + size_t(n_sums) * M * kClasses * sizeof(float) + 256;
+  // Extra Precision sums (M x N fp32 per linear that has a list) follow the class sums.
+  size_t ep_off = (psum_off + size_t(n_sums) * M * kClasses * sizeof(float) + 255) & ~size_t(255);
+  const size_t ep_begin = ep_off;
+  int n_ep = 0;
+  for (int i = 0; i < n_jobs; ++i) {
+    if (!jobs[i].ep_rows) continue;
+    if (++n_ep > kMaxEpJobs) return cudaErrorNotSupported;
+    ep_off += (size_t(M) * jobs[i].N * sizeof(float) + 255) & ~size_t(255);
+  }
+  const size_t ws_bytes = ep_off + 256;
   void* ws = nullptr;
   cudaError_t e = cudaSuccess;
   if (fixed) {
@@ -1028,6 +1033,20 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   for (int i = 0; i < n_jobs; ++i) {
     gp.lin[i].xf = wsb + layouts[lay_of[i]].off;
     gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * kClasses;
+  }
+  {
+    size_t off = ep_begin;
+    int k = 0;
+    for (int i = 0; i < n_jobs; ++i) {
+      const LinearJob& j = jobs[i];
+      if (!j.ep_rows) continue;
+      float* out = reinterpret_cast<float*>(wsb + off);
+      gp.lin[i].epc = out;
+      pp.ep[k++] = {j.ep_rows, j.ep_cols, static_cast<const __nv_bfloat16*>(j.x), out,
+                    static_cast<int>(j.N), static_cast<int>(j.K)};
+      off += (size_t(M) * j.N * sizeof(float) + 255) & ~size_t(255);
+    }
+    pp.n_ep = k;
   }
 
   // Stage layout: [128 rows x P0][128 rows x P1][M x KC bf16 activations].
@@ -1108,6 +1127,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
                  psum_base + size_t(i) * M * kClasses, sum_k[i]};
   }
   int prep_grid = std::max(n_sums * M, sms);
+  if (pp.n_ep > 0) prep_grid = 4 * sms;  // the Extra Precision gathers want many warps in flight
   prep_grid = std::min(prep_grid, 4 * sms);
   gemv_prep_kernel<CAP><<<prep_grid, 256, 0, stream>>>(pp);
   e = cudaGetLastError();
