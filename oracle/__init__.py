@@ -19,6 +19,9 @@ Python integers, written from the Matryoshka Quantization pages:
 * ``planes``   -- the dense r-bit plane layout the library stores slices in
                   (the layout is this library's own; the pages fix only that
                   lower widths are stored densely as r-bit integers).
+* ``chain``    -- a chained decoder stack over the sliced linears with a plain
+                  stand-in glue (RMSNorm, single-token attention, SwiGLU,
+                  residual), which the pages leave undefined.
 * ``matmul``   -- dequantize and y = x . W_r^T in float64, the element-wise
                   tolerance bound, and the per-layer-width (Mix'n'Match) stack
                   (same page, "Mix'n'Match and Interpolative Slicing").
