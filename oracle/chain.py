@@ -59,14 +59,18 @@ def silu(g: np.ndarray) -> np.ndarray:
 
 
 def chain_forward(h: np.ndarray, layers, d: int, dkv: int, head_dim: int, eps: float = 1e-6,
-                  trace: list | None = None) -> np.ndarray:
+                  trace: list | None = None, bound: list | None = None) -> np.ndarray:
     """Runs the layers in order on the residual stream h (M x d).
 
     layers: list of dicts with float64 weight matrices "qkv" ((d + 2 dkv) x d),
     "o" (d x d), "gate" and "up" (f x d), "down" (d x f). If `trace` is a
-    list, the residual stream after each layer is appended to it.
+    list, the residual stream after each layer is appended to it. If `bound`
+    is a list, the running sum over the layers so far of the two residual
+    linears' element-wise bounds 1e-3 (|a| |W_o|^T + |act| |W_down|^T) (the
+    per-linear accuracy bound of the decode path) is appended after each layer.
     """
     h = np.asarray(h, dtype=np.float64).copy()
+    acc = np.zeros_like(h)
     for L in layers:
         xn = to_bf16(rmsnorm(h, eps))
         qkv = xn @ L["qkv"].T
@@ -77,4 +81,7 @@ def chain_forward(h: np.ndarray, layers, d: int, dkv: int, head_dim: int, eps: f
         h = h1 + act @ L["down"].T
         if trace is not None:
             trace.append(h.copy())
+        if bound is not None:
+            acc = acc + 1e-3 * (np.abs(a) @ np.abs(L["o"]).T + np.abs(act) @ np.abs(L["down"]).T)
+            bound.append(acc.copy())
     return h

@@ -100,3 +100,25 @@ def test_pins_catch_a_dropped_residual():
             h = ch.to_bf16(ch.attention_single_token(xn @ L["qkv"].T, d, dkv, hd)) @ L["o"].T
         return h
     assert not np.array_equal(no_residual(h, [_zero_layer(d, dkv, f)]), h)
+
+
+def test_chain_bound_accumulates_the_residual_linears():
+    # one layer: the bound is 1e-3 (|a| |Wo|^T + |act| |Wdown|^T), and zero
+    # weights give a zero bound
+    d, dkv, f, hd = 16, 8, 32, 4
+    rng = np.random.default_rng(5)
+    h = rng.standard_normal((2, d))
+    b = []
+    ch.chain_forward(h, [_zero_layer(d, dkv, f)] * 2, d, dkv, hd, bound=b)
+    assert len(b) == 2 and not b[0].any() and not b[1].any()
+    L = {k: rng.standard_normal(v.shape) for k, v in _zero_layer(d, dkv, f).items()}
+    b = []
+    ch.chain_forward(h, [L, L], d, dkv, hd, bound=b)
+    xn = ch.to_bf16(ch.rmsnorm(h))
+    a = ch.to_bf16(ch.attention_single_token(xn @ L["qkv"].T, d, dkv, hd))
+    h1 = h + a @ L["o"].T
+    xn1 = ch.to_bf16(ch.rmsnorm(h1))
+    act = ch.to_bf16(ch.silu(xn1 @ L["gate"].T) * (xn1 @ L["up"].T))
+    want = 1e-3 * (np.abs(a) @ np.abs(L["o"]).T + np.abs(act) @ np.abs(L["down"]).T)
+    assert np.allclose(b[0], want, rtol=1e-12)
+    assert np.all(b[1] > b[0])
