@@ -419,6 +419,32 @@ def run_gpu(args, rank, world, local):
             per_width[f"r{r}"] = {"layers": nl, "us_per_layer": round(msr * 1000 / nl, 2),
                                   "GBps": round(stack.bytes_by_width[r] / (msr * 1e-3) / 1e9, 1)}
 
+        # Chained decode step (mq_chain_forward): each layer's output feeds the
+        # next through the stand-in glue, so a token is a chain of dependent
+        # launches; timed directly and replayed from a captured CUDA graph.
+        chain = None
+        if not args.no_chain and WORKLOAD == "mixnmatch_7b_stack" and len(stack.lins) == 5 * stack.layers:
+            D, Dkv, F, hd = 4096, 1024, 14336, 128
+            clayers = [(stack.widths[l], [(p, a, z) for (_, p, a, z, _, _, _) in stack.lins[5 * l:5 * l + 5]])
+                       for l in range(stack.layers)]
+            cplan = mq.ChainPlan(clayers, args.M, D, Dkv, F, hd)
+            cscratch = torch.empty(mq.chain_scratch_bytes(args.M, D, Dkv, F), dtype=torch.uint8, device=dev)
+            gen_h = torch.Generator(device=dev)
+            gen_h.manual_seed(77)
+            h_res = torch.randn((args.M, D), generator=gen_h, device=dev)
+            n_chain = max(3, args.steps // 4)
+            ms_direct = time_device(lambda: cplan.run(h_res, cscratch, False, stream), n_chain, 3, stream,
+                                    world, dev)
+            ms_graph = time_device(lambda: cplan.run(h_res, cscratch, True, stream), n_chain, 3, stream,
+                                   world, dev)
+            mq.device_status(stream)
+            chain = {"layers": stack.layers, "launches_per_token": 1 + 12 * stack.layers,
+                     "us_per_token_direct": round(ms_direct * 1000, 1),
+                     "us_per_token_graph": round(ms_graph * 1000, 1),
+                     "GBps_graph": round(stack.packed_bytes / (ms_graph * 1e-3) / 1e9, 1),
+                     "glue": "RMSNorm, single-token attention, SwiGLU, fp32 residual (stand-in)"}
+            del cscratch
+
         # end to end through the C ABI with host buffers: pinned x in, y out
         xs_host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in stack.x.items()}
         for k, v in xs_host.items():
@@ -470,6 +496,7 @@ def run_gpu(args, rank, world, local):
         "us_per_layer": round(ms * 1000 / stack.layers, 2),
         "tokens_per_s": round(args.M * world * 1000.0 / ms, 1),
         "per_width": per_width,
+        "chain": chain,
         "roofline": {
             "bound": "hbm",
             "achieved": round(achieved, 1),
@@ -570,6 +597,7 @@ def main(argv=None):
                     help="comma-separated per-layer widths; overrides --layers (small profiling stacks)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-chain", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--rows-only", action="store_true",
                     help="time only the separate rows (quantize, slice-pack, one decode linear, "

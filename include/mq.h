@@ -222,6 +222,47 @@ MQ_API mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_o
                            int n_lins, const int* widths, int n_layers,
                            int64_t M, void* stream);
 
+/*
+ * A chained decoder stack: each layer's output is the next layer's input, so
+ * one call is one token's decode step through n_layers dependent layers. The
+ * pages quantize the linears only (each layer at its own Mix'n'Match width)
+ * and define no glue between them; the stand-in glue per layer is
+ *   xn  = bf16(rmsnorm(h));  qkv = xn Wqkv^T;
+ *   a   = bf16(v of each query head's kv group)   (attention over a context
+ *         of one token: the softmax over a single score is 1);
+ *   h1  = h + a Wo^T;  xn1 = bf16(rmsnorm(h1));
+ *   act = bf16(silu(xn1 Wgate^T) * (xn1 Wup^T));  h = h1 + act Wdown^T,
+ * with rmsnorm(v) = v / sqrt(mean(v^2) + 1e-6) (no learned scale),
+ * silu(g) = g / (1 + exp(-g)), the residual stream h in fp32 and every
+ * linear run by the decode path of mq_linear at the layer's width.
+ *   layers  : n_layers host descriptors; packed/alpha/zero index 0..4 =
+ *             qkv ((D + 2 Dkv) x D), o (D x D), gate (F x D), up (F x D),
+ *             down (D x F), each packed at width r.
+ *   h       : M x D fp32 (device), the residual stream in and out.
+ *   D, Dkv, F, head_dim : model width, key/value width, MLP width, head
+ *             size; D and F multiples of 128, head_dim dividing Dkv, and
+ *             D / head_dim a multiple of Dkv / head_dim.
+ *   scratch : mq_chain_scratch_bytes(M, D, Dkv, F) bytes (device), 256-byte
+ *             aligned, owned by the caller; the chain allocates nothing.
+ *   flags   : MQ_CHAIN_GRAPH to capture the call into a CUDA graph on its
+ *             second identical call (same stream, pointers and sizes) and
+ *             replay it from then on; the first call runs directly. Graphs
+ *             are freed by mq_release_workspace. Needs a stream other than
+ *             the legacy default stream (there the flag is ignored).
+ * Requires 1 <= M <= 32.
+ */
+typedef struct mq_chain_layer {
+  int r;
+  const void* packed[5];
+  const float* alpha[5];
+  const float* zero[5];
+} mq_chain_layer;
+#define MQ_CHAIN_GRAPH 1
+MQ_API size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F);
+MQ_API mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
+                                  int64_t Dkv, int64_t F, int64_t head_dim, float* h,
+                                  void* scratch, size_t scratch_bytes, int flags, void* stream);
+
 /* Bytes of the device array that mq_linear_noalloc works in (1.25 MiB). */
 #define MQ_NOALLOC_SCRATCH_BYTES (1280u * 1024u)
 

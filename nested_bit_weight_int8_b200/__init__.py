@@ -36,6 +36,14 @@ class LinearDesc(ctypes.Structure):
                 ("N", _i64), ("K", _i64)]
 
 
+class ChainLayer(ctypes.Structure):
+    """mq_chain_layer: one layer of a chained stack (qkv, o, gate, up, down at width r)."""
+    _fields_ = [("r", _int), ("packed", _vp * 5), ("alpha", _vp * 5), ("zero", _vp * 5)]
+
+
+MQ_CHAIN_GRAPH = 1
+
+
 def _sig(name, res, args):
     f = getattr(_lib, name)
     f.restype = res
@@ -60,6 +68,10 @@ _ovf_rows = _sig("mq_ep_overflow_rows", _int, [_vp, _i64, _i64, _int, _vp, _vp])
 _ovf_cols = _sig("mq_ep_overflow_cols", _int, [_vp, _i64, _i64, _int, _vp, _vp, _vp])
 _linear_ep = _sig("mq_linear_ep", _int,
                   [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _vp])
+_chain_bytes = _sig("mq_chain_scratch_bytes", ctypes.c_size_t, [_i64, _i64, _i64, _i64])
+_chain = _sig("mq_chain_forward", _int,
+              [ctypes.POINTER(ChainLayer), _int, _i64, _i64, _i64, _i64, _i64, _vp, _vp,
+               ctypes.c_size_t, _int, _vp])
 _linear_noalloc = _sig("mq_linear_noalloc", _int,
                       [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
 _device_status = _sig("mq_device_status", _int, [_vp])
@@ -70,7 +82,8 @@ EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8"
             "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
             "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc",
             "mq_quantize_int8_clipped", "mq_linear_container", "mq_ep_overflow_rows",
-            "mq_ep_overflow_cols", "mq_linear_ep")
+            "mq_ep_overflow_cols", "mq_linear_ep", "mq_chain_scratch_bytes",
+            "mq_chain_forward")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -161,6 +174,33 @@ def linear_ep(x, M: int, K: int, packed, alpha, zero, N: int, r: int, row_ptr, c
     """Eq. 8 (Extra Precision) product: the Eq. 6 planes plus the sparse list."""
     _check(_linear_ep(_ptr(x), M, K, _ptr(packed), _ptr(alpha), _ptr(zero), N, r, _ptr(row_ptr),
                       _ptr(cols), _ptr(y), _stream(stream)))
+
+
+def chain_scratch_bytes(M: int, D: int, Dkv: int, F: int) -> int:
+    return int(_chain_bytes(M, D, Dkv, F))
+
+
+class ChainPlan:
+    """Host descriptors of a chained stack, built once and reused. `layers` is
+    a list of (r, [qkv, o, gate, up, down]) with each linear a (packed, alpha,
+    zero) triple of device tensors."""
+
+    def __init__(self, layers, M: int, D: int, Dkv: int, F: int, head_dim: int):
+        self.M, self.D, self.Dkv, self.F, self.hd = M, D, Dkv, F, head_dim
+        self.n = len(layers)
+        self.arr = (ChainLayer * self.n)()
+        for i, (r, lins) in enumerate(layers):
+            self.arr[i].r = r
+            for j, (p, a, z) in enumerate(lins):
+                self.arr[i].packed[j] = _ptr(p)
+                self.arr[i].alpha[j] = _ptr(a)
+                self.arr[i].zero[j] = _ptr(z)
+
+    def run(self, h, scratch, graph: bool = False, stream=None) -> None:
+        """One decode step through every layer: h (M x D fp32) in place."""
+        nbytes = scratch.numel() * scratch.element_size()
+        _check(_chain(self.arr, self.n, self.M, self.D, self.Dkv, self.F, self.hd, _ptr(h),
+                      _ptr(scratch), nbytes, MQ_CHAIN_GRAPH if graph else 0, _stream(stream)))
 
 
 def linear_noalloc(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=None) -> None:

@@ -256,6 +256,46 @@ mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed, 
   return MQ_OK;
 }
 
+size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
+  if (M < 1 || M > 32 || D < 128 || Dkv < 1 || F < 128) return 0;
+  return chain_scratch_bytes(M, D, Dkv, F);
+}
+
+mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
+                           int64_t Dkv, int64_t F, int64_t head_dim, float* h, void* scratch,
+                           size_t scratch_bytes, int flags, void* stream) {
+  g_last_error.clear();
+  const char* who = "mq_chain_forward";
+  if (!layers || !h || !scratch) return fail(MQ_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (n_layers < 1) return fail(MQ_ERR_INVALID_ARG, "%s: n_layers must be >= 1", who);
+  if (M < 1 || M > 32) return fail(MQ_ERR_INVALID_ARG, "%s: M must be in [1, 32]", who);
+  if (D < 128 || D % 128 || F < 128 || F % 128) return fail(MQ_ERR_INVALID_ARG, "%s: D and F must be positive multiples of 128", who);
+  if (head_dim < 1 || Dkv < head_dim || Dkv % head_dim || D % head_dim || (D / head_dim) % (Dkv / head_dim))
+    return fail(MQ_ERR_INVALID_ARG, "%s: head_dim must divide Dkv and D, and D / head_dim be a multiple of Dkv / head_dim", who);
+  if (D > (int64_t(1) << 20) || F > (int64_t(1) << 20) || Dkv > (int64_t(1) << 20))
+    return fail(MQ_ERR_UNSUPPORTED, "%s: dimensions too large", who);
+  if (flags & ~MQ_CHAIN_GRAPH) return fail(MQ_ERR_INVALID_ARG, "%s: unknown flags", who);
+  if (!aligned(h, 4) || !aligned(scratch, 256)) return fail(MQ_ERR_INVALID_ARG, "%s: h must be 4-byte and scratch 256-byte aligned", who);
+  if (scratch_bytes < chain_scratch_bytes(M, D, Dkv, F)) return fail(MQ_ERR_INVALID_ARG, "%s: scratch smaller than mq_chain_scratch_bytes", who);
+  const int64_t nout[5] = {D + 2 * Dkv, D, F, F, D};
+  const int64_t nin[5] = {D, D, D, D, F};
+  for (int l = 0; l < n_layers; ++l) {
+    const mq_chain_layer& L = layers[l];
+    for (int i = 0; i < 5; ++i) {
+      char w[64];
+      std::snprintf(w, sizeof(w), "%s[layer %d, linear %d]", who, l, i);
+      // a 16-byte-aligned stand-in for x: the chain's own bf16 buffers
+      mq_status st = check_linear(w, scratch, M, nin[i], L.packed[i], L.alpha[i], L.zero[i], nout[i], L.r, h);
+      if (st != MQ_OK) return st;
+    }
+  }
+  cudaError_t e = run_chain(layers, n_layers, static_cast<int>(M), static_cast<int>(D), static_cast<int>(Dkv),
+                            static_cast<int>(F), static_cast<int>(head_dim), h, scratch,
+                            (flags & MQ_CHAIN_GRAPH) != 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return MQ_OK;
+}
+
 mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, int n_lins,
                            const int* widths, int n_layers, int64_t M, void* stream) {
   g_last_error.clear();
@@ -315,6 +355,7 @@ mq_status mq_release_workspace(void) {
   }
   g_workspaces.clear();
   cudaSetDevice(cur);
+  release_chain_graphs();
   return MQ_OK;
 }
 

@@ -1181,6 +1181,13 @@ size_t gemv_scratch_bytes(const LinearJob& job, int M) {
   return xf + size_t(M) * kClasses * sizeof(float) + 256;
 }
 
+cudaError_t run_gemv_fixed_n(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream,
+                             const FixedScratch& scratch) {
+  if (n_jobs < 1 || n_jobs > 8 || M < 1 || M > 32) return cudaErrorInvalidValue;
+  if (n_jobs == 1) return run_gemv_cap<1>(jobs, 1, M, stream, &scratch);
+  return run_gemv_cap<8>(jobs, n_jobs, M, stream, &scratch);
+}
+
 cudaError_t run_gemv_fixed(const LinearJob& job, int M, cudaStream_t stream,
                            const FixedScratch& scratch) {
   if (M < 1 || M > 32) return cudaErrorInvalidValue;

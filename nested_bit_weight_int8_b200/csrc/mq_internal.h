@@ -113,6 +113,17 @@ cudaError_t launch_ovf_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32
 cudaError_t launch_ovf_cols(const uint8_t* q, int64_t N, int64_t K, int r, const int32_t* row_ptr,
                             uint16_t* cols, cudaStream_t stream, int sms);
 
+// Decode path for up to 8 linears on caller-provided scratch.
+cudaError_t run_gemv_fixed_n(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream,
+                             const FixedScratch& scratch);
+
+// Chained decoder stack (mq_chain_forward): scratch bytes, and the run, with
+// graph capture and replay of repeated identical calls when `use_graph`.
+size_t chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F);
+cudaError_t run_chain(const struct mq_chain_layer* layers, int n_layers, int M, int D, int Dkv, int F,
+                      int hd, float* h, void* scratch, bool use_graph, cudaStream_t stream);
+void release_chain_graphs();
+
 // Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
 // cudaErrorNotSupported for shapes it does not serve (nothing launched).
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);
