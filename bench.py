@@ -543,11 +543,16 @@ def _profile_traffic():
         return None
 
 
+# The sources the stack's decode kernels (gemv_prep_kernel, gemv_streamk_kernel)
+# are built from: their DRAM counters stay valid while these are unchanged.
+KERNEL_SOURCES = ("gemv.cu", "mq_device.cuh", "mq_internal.h", "tensor_map.cu")
+
+
 def _kernel_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nested_bit_weight_int8_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

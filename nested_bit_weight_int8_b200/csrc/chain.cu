@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "../../include/mq.h"
+#include "mq_device.cuh"
 #include "mq_internal.h"
 
 namespace mq {
@@ -39,6 +40,8 @@ rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ add, float
                __nv_bfloat16* __restrict__ xn, int D) {
   __shared__ float red[kGlueThreads / 32];
   __shared__ float s_inv;
+  pdl_launch_dependents();
+  pdl_wait_primary();
   const int m = blockIdx.x, tid = threadIdx.x;
   const float* hr = h + int64_t(m) * D;
   const float* ar = add ? add + int64_t(m) * D : nullptr;
@@ -69,6 +72,8 @@ rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ add, float
 __global__ void __launch_bounds__(kGlueThreads)
 attn_one_token_kernel(const float* __restrict__ qkv, __nv_bfloat16* __restrict__ a, int M, int D,
                       int Dkv, int hd) {
+  pdl_launch_dependents();
+  pdl_wait_primary();
   const int per_group = (D / hd) / (Dkv / hd);
   const int nq = D + 2 * Dkv;
   const int64_t total = int64_t(M) * D;
@@ -84,6 +89,8 @@ attn_one_token_kernel(const float* __restrict__ qkv, __nv_bfloat16* __restrict__
 __global__ void __launch_bounds__(kGlueThreads)
 swiglu_kernel(const float* __restrict__ g, const float* __restrict__ u, __nv_bfloat16* __restrict__ act,
               int64_t total) {
+  pdl_launch_dependents();
+  pdl_wait_primary();
   for (int64_t i = int64_t(blockIdx.x) * kGlueThreads + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * kGlueThreads) {
     const float gv = g[i];
@@ -153,8 +160,11 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
   cudaError_t e;
   // xn = bf16(rmsnorm(h)) for the first layer; later layers get it from the
   // previous layer's last norm
-  rmsnorm_kernel<<<M, kGlueThreads, 0, s>>>(c.h, nullptr, nullptr, bf(L.xn), D);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const float* no_add = nullptr;
+  float* no_out = nullptr;
+  e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(c.h), no_add,
+                 no_out, bf(L.xn), D);
+  if (e != cudaSuccess) return e;
   for (int l = 0; l < c.n_layers; ++l) {
     const mq_chain_layer& Ly = c.layers[l];
     auto job = [&](int which, const void* x, int64_t N, int64_t K, float* y) {
@@ -171,23 +181,26 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
     };
     LinearJob jq = job(0, bf(L.xn), D + 2 * Dkv, D, fp(L.qkv));
     if ((e = run_gemv_fixed_n(&jq, 1, M, s, fx)) != cudaSuccess) return e;
-    attn_one_token_kernel<<<glue_grid(int64_t(M) * D, sms), kGlueThreads, 0, s>>>(fp(L.qkv), bf(L.a), M, D,
-                                                                               Dkv, c.hd);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(attn_one_token_kernel, dim3(glue_grid(int64_t(M) * D, sms)), dim3(kGlueThreads), 0, s,
+                   static_cast<const float*>(fp(L.qkv)), bf(L.a), M, D, Dkv, c.hd);
+    if (e != cudaSuccess) return e;
     LinearJob jo = job(1, bf(L.a), D, D, fp(L.o));
     if ((e = run_gemv_fixed_n(&jo, 1, M, s, fx)) != cudaSuccess) return e;
-    rmsnorm_kernel<<<M, kGlueThreads, 0, s>>>(c.h, fp(L.o), fp(L.h1), bf(L.xn1), D);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(c.h),
+                   static_cast<const float*>(fp(L.o)), fp(L.h1), bf(L.xn1), D);
+    if (e != cudaSuccess) return e;
     LinearJob jgu[2] = {job(2, bf(L.xn1), F, D, fp(L.g)), job(3, bf(L.xn1), F, D, fp(L.u))};
     if ((e = run_gemv_fixed_n(jgu, 2, M, s, fx)) != cudaSuccess) return e;
-    swiglu_kernel<<<glue_grid(int64_t(M) * F, sms), kGlueThreads, 0, s>>>(fp(L.g), fp(L.u), bf(L.act),
-                                                                       int64_t(M) * F);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(swiglu_kernel, dim3(glue_grid(int64_t(M) * F, sms)), dim3(kGlueThreads), 0, s,
+                   static_cast<const float*>(fp(L.g)), static_cast<const float*>(fp(L.u)), bf(L.act),
+                   int64_t(M) * F);
+    if (e != cudaSuccess) return e;
     LinearJob jd = job(4, bf(L.act), D, F, fp(L.dn));
     if ((e = run_gemv_fixed_n(&jd, 1, M, s, fx)) != cudaSuccess) return e;
     // h = h1 + down, and the next layer's normalized input
-    rmsnorm_kernel<<<M, kGlueThreads, 0, s>>>(fp(L.h1), fp(L.dn), c.h, bf(L.xn), D);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(fp(L.h1)),
+                   static_cast<const float*>(fp(L.dn)), c.h, bf(L.xn), D);
+    if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }

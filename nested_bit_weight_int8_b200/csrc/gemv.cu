@@ -529,6 +529,9 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   uint8_t* stages = base + kHeaderBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
+  // The next kernel in the stream may be scheduled once every CTA of this
+  // grid is resident; it waits for this grid's completion before it reads.
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -712,7 +715,11 @@ static_assert(sizeof(PrepParams<kGemvMaxLinears>) <= 32764, "prep kernel paramet
 // blocks that several CTAs add into.
 template <int CAP>
 __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ PrepParams<CAP> p) {
+  // The decode kernel may start now (its weight boxes do not depend on this
+  // grid); this grid itself may have started before its predecessor in the
+  // stream finished, so it waits for it before touching memory.
   pdl_launch_dependents();
+  pdl_wait_primary();
   const int M = p.M;
   // (1) class sums: one CTA per (sum job, batch row)
   if (blockIdx.x < p.n_sum * M) {
@@ -1129,8 +1136,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   int prep_grid = std::max(n_sums * M, sms);
   if (pp.n_ep > 0) prep_grid = 4 * sms;  // the Extra Precision gathers want many warps in flight
   prep_grid = std::min(prep_grid, 4 * sms);
-  gemv_prep_kernel<CAP><<<prep_grid, 256, 0, stream>>>(pp);
-  e = cudaGetLastError();
+  e = launch_pdl(gemv_prep_kernel<CAP>, dim3(prep_grid), dim3(256), 0, stream, pp);
   if (e != cudaSuccess) return e;
 
   gp.n_lin = n_jobs;

@@ -55,6 +55,25 @@ inline int decode_kind(const LinearJob& j) {
   return j.src == kContainer ? 10 : 11;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while its predecessor in the stream finishes, so it must execute
+// griddepcontrol.wait before touching any memory the predecessor may use.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Per-(device, stream) scratch owned by the library.
 struct Workspace {
   void* ptr = nullptr;
