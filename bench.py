@@ -348,6 +348,13 @@ def rows_timings(dev, stream):
                 "us": round(us, 2), "TFLOPs": round(tf, 1),
                 "frac_of_bf16_peak": round(tf / bf16_peak, 3)}
             del p_p
+        # the same product sliced on load from the container (Eq. 6 at r = 4, Eq. 8 at r = 2)
+        for r, clamp, tag in ((4, True, "eq6"), (2, False, "eq8")):
+            us = timed(lambda: mq.linear_container(xm, m, k_p, q_p, a_p, z_p, n_p, r, clamp, ym, stream),
+                       reps=5)
+            tf = 2 * m * n_p * k_p / us / 1e6
+            out[f"prefill_container_{name}_r{r}_{tag}_M{m}"] = {
+                "us": round(us, 2), "TFLOPs": round(tf, 1), "frac_of_bf16_peak": round(tf / bf16_peak, 3)}
         del q_p, xm, ym
     torch.cuda.synchronize()
     return out

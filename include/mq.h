@@ -153,9 +153,10 @@ MQ_API mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* pack
  *   y[m,n] = sum_k x[m,k] * alpha_n * (code[n,k] * 2^s - z_n).
  * It streams 8 bits per weight: it saves the planes' storage, not bandwidth.
  *   q : N x K uint8 container (row pitch K bytes), 16-byte aligned.
- *   Other arguments and the accuracy bound as mq_linear. Requires
- *   1 <= M <= 32 (the decode path; larger M returns MQ_ERR_UNSUPPORTED),
- *   K % 128 == 0, clamp in {0, 1}. At r = 8 both forms are the container.
+ *   Other arguments and the accuracy bound as mq_linear: M <= 32 runs the
+ *   decode GEMV, larger M the prefill GEMM, both slicing while they decode.
+ *   Requires K % 128 == 0, clamp in {0, 1}. At r = 8 both forms are the
+ *   container.
  */
 MQ_API mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t* q,
                                      const float* alpha, const float* zero, int64_t N, int r,

@@ -200,9 +200,16 @@ mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t
   mq_status st = check_linear("mq_linear_container", x, M, K, q, alpha, zero, N, r, y);
   if (st != MQ_OK) return st;
   if (clamp != 0 && clamp != 1) return fail(MQ_ERR_INVALID_ARG, "mq_linear_container: clamp must be 0 or 1");
-  if (M > 32) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_container: M must be <= 32 (decode path)");
   LinearJob job{x, q, alpha, zero, y, N, K, r, clamp ? kContainer : kContainerEP};
-  cudaError_t e = run_gemv(&job, 1, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M <= 32) {
+    e = run_gemv(&job, 1, static_cast<int>(M), s);
+  } else {
+    if (M > (int64_t(1) << 24)) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_container: M too large");
+    e = run_gemm(job, static_cast<int>(M), s);
+  }
+  if (e == cudaErrorNotSupported) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_container: shape not served by this build");
   if (e != cudaSuccess) return cuda_fail(e, "mq_linear_container");
   return MQ_OK;
 }

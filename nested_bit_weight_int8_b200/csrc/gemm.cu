@@ -120,9 +120,25 @@ __device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo
 // A operand in tensor memory expects). `p0` / `p1` point at this row's 32-code
 // slice of plane 0 / plane 1 in shared memory. Plane word layout: local code
 // u of a width-b word sits at bit 16*(u%2) + b*(u/2) (b < 8), at 8u for b = 8.
+// R = 10 / 11: the int8 container sliced on load by Eq. 6 / Eq. 8 (runtime
+// width r): code = min(q + 2^(s-1), 255) >> s, or (q + 2^(s-1)) >> s, on the
+// two 16-bit halves at once (h2 = 2^(s-1) in both halves, kmask the code's
+// bits in both halves after the shift by s).
 template <int R>
-__device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[16]) {
-  if constexpr (R == 2) {
+__device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[16],
+                                         uint32_t h2 = 0, uint32_t kmask = 0, int sh = 0) {
+  if constexpr (R == 10 || R == 11) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p0);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      // codes 2j, 2j+1 are bytes (0, 1) or (2, 3) of word j / 2
+      const uint32_t t = __byte_perm(w[j / 2], 0u, (j % 2 == 0) ? 0x4140u : 0x4342u);
+      const uint32_t u = (R == 10) ? __viaddmin_u16x2(t, h2, 0x00FF00FFu) : t + h2;
+      v[j] = exact_pair((u >> sh) & kmask);
+    }
+  } else if constexpr (R == 2) {
     const uint2 a = *reinterpret_cast<const uint2*>(p0);
     const uint32_t w[2] = {a.x, a.y};
 #pragma unroll
@@ -214,7 +230,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       int issued = 0;
       // plane 0: 8*b0 bytes (64 codes) per row; plane 1: the 16-byte chunk
       // that holds the stage's codes (64 codes at b1 = 2, 128 at b1 = 1)
-      constexpr uint32_t b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
+      constexpr uint32_t b0 = (R == 8 || R >= 10) ? 8 : (R == 4 || R == 6) ? 4 : 2;
       const uint32_t p0_bytes = 128u * 8u * b0;
       const uint32_t p1_bytes = (R == 3 || R == 6) ? 128u * 16u : 0u;
       for (int it = 0; it < n_k; ++it, ++issued) {
@@ -280,7 +296,11 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
     const int grp = (warp - kDecodeWarp0) >> 3;      // which stages: it % 2 == grp
     const int row = 32 * q + lane;             // weight row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    constexpr int b0 = (R == 8) ? 8 : (R == 4 || R == 6) ? 4 : 2;
+    constexpr int b0 = (R == 8 || R >= 10) ? 8 : (R == 4 || R == 6) ? 4 : 2;
+    // slice-on-load constants (container kinds 10, 11)
+    const int cs = 8 - p.r;
+    const uint32_t ch2 = (R >= 10) ? (1u << (cs - 1)) * 0x10001u : 0u;
+    const uint32_t ckm = (R >= 10) ? ((1u << (R == 10 ? p.r : p.r + 1)) - 1u) * 0x10001u : 0u;
     constexpr int b1 = (R == 3) ? 1 : (R == 6) ? 2 : 0;
     bool ok = true;
     for (int it = grp; it < n_k; it += 2) {
@@ -303,7 +323,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       const uint8_t* r1 = st + p.off_p1 + row * 16 +
                           (b1 == 1 ? (it % 2) * 8 + h * 4 : h * 8);
       uint32_t v[16];
-      decode32<R>(r0, r1, v);
+      decode32<R>(r0, r1, v, ch2, ckm, cs);
       tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();
@@ -321,7 +341,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       float A = 0.f, B = 0.f;
       if (row_ok) {
         const float a = __ldg(p.alpha + n);
-        A = a * static_cast<float>(1 << (8 - R));
+        A = a * static_cast<float>(1 << (8 - (R >= 10 ? p.r : R)));
         B = a * __ldg(p.zero + n);
       }
 #pragma unroll 1
@@ -381,8 +401,9 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   if (M < 1 || job.K % kBK != 0 || job.N < 1) return cudaErrorNotSupported;
   if ((job.N + kBN - 1) / kBN > 0x7FFFFFFF || (M + kBM - 1) / kBM > 65535) return cudaErrorNotSupported;
   int b0, b1;
-  plane_widths(job.r, b0, b1);
+  job_planes(job, b0, b1);
   if (b0 == 0) return cudaErrorInvalidValue;
+  if (job.ep_rows) return cudaErrorNotSupported;  // Extra Precision lists serve the decode path only
 
   static thread_local GemmParams gp;
   cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, true);
@@ -429,7 +450,9 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
 
   const dim3 grid(static_cast<unsigned>((job.N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
-  switch (job.r) {
+  switch (decode_kind(job)) {
+    case 10: return launch_gemm_r<10>(gp, grid, smem, stream);
+    case 11: return launch_gemm_r<11>(gp, grid, smem, stream);
     case 8: return launch_gemm_r<8>(gp, grid, smem, stream);
     case 6: return launch_gemm_r<6>(gp, grid, smem, stream);
     case 4: return launch_gemm_r<4>(gp, grid, smem, stream);

@@ -117,7 +117,6 @@ def test_linear_container_rejects():
         ((F, 1, 96, F, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),     # K % 128
         ((F, 1, 256, F + 4, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),  # misaligned q
         ((F, 1, 256, None, F, F, 64, 4, 0, F), mq.MQ_ERR_INVALID_ARG),   # null q
-        ((F, 33, 256, F, F, F, 64, 4, 1, F), mq.MQ_ERR_UNSUPPORTED),   # prefill batch
     ]
     for c, want in bad:
         assert mq.raw_status("mq_linear_container", *c, None) == want, c

@@ -103,3 +103,51 @@ def test_container_matches_planes_within_bound():
     wr = oracle.dequant_slice(q, a, z, r)
     tol = oracle.tolerance(x_vals, wr)
     assert np.all(np.abs(yc - yp.cpu().numpy()) <= 2 * tol)
+
+
+def _prefill_case(law, n, k, seed, r, clamp, m, xseed, rows=None):
+    _, w_vals = weights(law, n, k, seed)
+    q, a, z = oracle.quantize_minmax(w_vals)
+    x_bits = synth.activations(m, k, xseed)
+    x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
+    y = gpu_linear_container(x_bits, q, a, z, r, clamp)
+    label = f"container prefill {law} {n}x{k} r={r} clamp={clamp} M={m}"
+    if rows is None:
+        return check_linear(y, x_vals, oracle.dequant_slice(q, a, z, r, clamp=clamp), label)
+    # rows are quantized independently, so the oracle on a row sample is exact
+    return check_linear(y[:, rows], x_vals, oracle.dequant_slice(q[rows], a[rows], z[rows], r, clamp=clamp),
+                        label + " (sampled rows)")
+
+
+@pytest.mark.parametrize("clamp", [True, False])
+@pytest.mark.parametrize("r", [8, 6, 4, 3, 2])
+@pytest.mark.parametrize("m,n,k", [(33, 300, 1024), (160, 1000, 640), (257, 129, 4224)])
+def test_container_prefill_ragged(m, n, k, r, clamp):
+    _prefill_case("t", n, k, 31 + n, r, clamp, m, 37 + m)
+
+
+@pytest.mark.parametrize("clamp", [True, False])
+@pytest.mark.parametrize("r", [4, 2])
+def test_container_prefill_9b_up_sampled_rows(r, clamp):
+    n, k = 14336, 3584
+    rng = np.random.default_rng(r)
+    rows = np.unique(np.concatenate([rng.choice(n, size=48, replace=False), [0, 127, 128, n - 1]]))
+    _prefill_case("gauss", n, k, 500, r, clamp, 2048, 600, rows=rows)
+
+
+def test_container_prefill_every_byte():
+    # every container value in every row, both forms, through the GEMM
+    n, k, m = 256, 1024, 64
+    rng = np.random.default_rng(3)
+    q = np.tile(np.arange(256, dtype=np.uint8), (n, 4))
+    for i in range(n):
+        rng.shuffle(q[i])
+    a = (rng.uniform(0.5, 2.0, n) * 1e-3).astype(np.float32)
+    z = rng.uniform(0.0, 255.0, n).astype(np.float32)
+    x_bits = synth.activations(m, k, 5)
+    x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
+    for r in (6, 4, 3, 2):
+        for clamp in (True, False):
+            y = gpu_linear_container(x_bits, q, a, z, r, clamp)
+            check_linear(y, x_vals, oracle.dequant_slice(q, a, z, r, clamp=clamp),
+                         f"prefill bytes r={r} clamp={clamp}")
