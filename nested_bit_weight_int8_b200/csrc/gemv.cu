@@ -28,8 +28,9 @@
 // sum to O_m = sum_k x[m,k] off(k), which depends only on k mod 16 and is
 // removed in the epilogue from per-class activation sums computed once:
 //   y = A_n (acc - O_m) - B_n Sx_m,  A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n.
-// Offsets stay <= 384, so fp32 partial sums stay small (accuracy), and
-// two codes are decoded per shift+LOP3 pair (issue budget at r = 2).
+// Offsets stay <= 272 (none at r = 8, whose bytes go through fp32 exactly),
+// so fp32 partial sums stay small (accuracy), and two codes are decoded per
+// shift+LOP3 pair (issue budget at r = 2).
 //
 // Slicing on load. A linear may also stream the int8 container itself (the
 // r = 8 plane) and slice each byte while decoding, so one stored matrix serves
@@ -188,6 +189,16 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   return d;
 }
 
+// Two bytes of w (chosen by the byte_perm selectors, which put the byte under
+// the exponent of 2^23) as an exact bf16x2 pair of integers 0..255.
+__device__ __forceinline__ uint32_t bytes_bf16x2(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
+  const float lo = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - 8388608.0f;
+  const float hi = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - 8388608.0f;
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 // The pair of 2-bit codes at half-word position P (0, 2, ..., 14) of a plane
 // word as bf16x2. Positions 0-4 need no shift, 6-10 one shift by 6, 12-14 one
 // by 12, so a word costs two shifts and eight LOP3s. The code lands at bit
@@ -244,16 +255,13 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
     x0 = and_or(shift_to<8 * HF - 3>(w), kMaskP3b4, kMag16);
     x1 = and_or(shift_to<8 * HF + 1>(w), kMaskP3b4, kMag16);
   } else if constexpr (R == 8) {
-    // bytes c0..c3 of one word; registers pair (c0, c2) and (c1, c3):
-    // low nibble -> 128 + l (bits 0-3), high nibble -> 256 + 16h (bits 3-6)
+    // bytes c0..c3 of one word; registers pair (c0, c2) and (c1, c3). A byte
+    // has 8 significant bits, one more than a bf16 mantissa holds under a
+    // magic exponent, so it goes through fp32: 2^23 + c minus 2^23 is c, and
+    // its conversion to bf16 is exact. No offset remains.
     const uint32_t w = lo[2 * Q + HF];
-    if constexpr (PLANE == 0) {
-      x0 = and_or(w, kMaskP0b4, kMag128);
-      x1 = and_or(w >> 8, kMaskP0b4, kMag128);
-    } else {
-      x0 = and_or(w >> 1, kMaskP3b4, kMag256);
-      x1 = and_or(w >> 9, kMaskP3b4, kMag256);
-    }
+    x0 = bytes_bf16x2(w, 0x7440u, 0x7442u);
+    x1 = bytes_bf16x2(w, 0x7441u, 0x7443u);
   } else if constexpr (R == 3) {
     // high 1-bit plane (weight 4), word = 32 codes; pairs P = 4(Q%4)+2HF, +1 at
     // half-bit P; one shift puts the group's 4 pairs at bits 3..6 (64/32/16/8 + 4h)
@@ -283,7 +291,7 @@ __device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses
   const float cont = static_cast<float>(1 << (dk == 10 ? r : r + 1));
 #pragma unroll
   for (int i = 0; i < kClasses; ++i) {
-    c[i] = dk >= 10 ? cont : r == 8 ? 384.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
+    c[i] = dk >= 10 ? cont : r == 8 ? 0.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
   }
 }
 
@@ -303,8 +311,8 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
     const uint32_t a = xaddr[nt] + static_cast<uint32_t>(gbase + Q) * xstep[nt];
     xb[nt] = *reinterpret_cast<const uint4*>(smem + a);
   }
-  // two operand planes for r = 3, 6 (low/high bit planes) and r = 8 (low/high nibbles)
-  constexpr int NPL = (Geo<R>::b1 != 0 || R == 8) ? 2 : 1;
+  // two operand planes for r = 3, 6 (low/high bit planes)
+  constexpr int NPL = (Geo<R>::b1 != 0) ? 2 : 1;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
