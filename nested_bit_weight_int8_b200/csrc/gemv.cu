@@ -940,17 +940,17 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
 
 // Relative cost of one unit of each width, for cutting the CTA ranges. A unit
 // always holds the same plane bytes per row (two planes hold 1.5x), while the
-// decode and MMA work grows with the codes in it: measured per-unit times of
-// single-width stacks on B200 at M = 1 put r = 2 at about 1.6x and r = 4 at
-// about 1.1x an r = 8 unit; r = 3 and 6 are estimated from their planes.
+// decode and MMA work grows with the codes in it: per-unit times of
+// single-width stacks on B200 at M = 1 put r = 4 at about 1.26x and r = 2 at
+// about 1.93x an r = 8 unit; r = 3 and 6 are scaled from their planes.
 int64_t unit_cost(const LinearJob& j) {
   switch (decode_kind(j)) {
     case 8: return 100;
-    case 4: return 108;
-    case 2: return 157;
-    case 6: return 170;
+    case 4: return 126;
+    case 2: return 193;
+    case 6: return 183;
     case 10: case 11: return 110;  // one 8-bit plane, one MMA per 16 codes, more decode work
-    default: return 280;  // 3
+    default: return 301;  // 3
   }
 }
 
