@@ -40,6 +40,8 @@ mq_status cuda_fail(cudaError_t e, const char* where) {
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+
 bool valid_r(int r) { return r == 8 || r == 6 || r == 4 || r == 3 || r == 2; }
 
 }  // namespace
@@ -119,6 +121,7 @@ size_t mq_packed_bytes(int64_t N, int64_t K, int r) {
 
 mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K, uint8_t* q,
                            float* alpha, float* zero, void* stream) {
+  TraceRange trace_("mq_quantize_int8");
   g_last_error.clear();
   if (!w || !q || !alpha || !zero) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: null pointer");
   if (dtype != MQ_F32 && dtype != MQ_BF16) return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8: dtype must be MQ_F32 or MQ_BF16");
@@ -135,6 +138,7 @@ mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K, uint8
 mq_status mq_quantize_int8_clipped(const void* w, int dtype, int64_t N, int64_t K,
                                    const float* gamma, const float* beta, uint8_t* q, float* alpha,
                                    float* zero, void* stream) {
+  TraceRange trace_("mq_quantize_int8_clipped");
   g_last_error.clear();
   if (!w || !gamma || !beta || !q || !alpha || !zero)
     return fail(MQ_ERR_INVALID_ARG, "mq_quantize_int8_clipped: null pointer");
@@ -150,6 +154,7 @@ mq_status mq_quantize_int8_clipped(const void* w, int dtype, int64_t N, int64_t 
 }
 
 mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* packed, void* stream) {
+  TraceRange trace_("mq_slice_pack");
   g_last_error.clear();
   if (!q || !packed) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: null pointer");
   if (!valid_r(r)) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: r=%d not in {8,6,4,3,2}", r);
@@ -176,6 +181,7 @@ static mq_status check_linear(const char* who, const void* x, int64_t M, int64_t
 
 mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed, const float* alpha,
                     const float* zero, int64_t N, int r, float* y, void* stream) {
+  TraceRange trace_("mq_linear");
   g_last_error.clear();
   mq_status st = check_linear("mq_linear", x, M, K, packed, alpha, zero, N, r, y);
   if (st != MQ_OK) return st;
@@ -196,6 +202,7 @@ mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed, con
 mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t* q,
                               const float* alpha, const float* zero, int64_t N, int r, int clamp,
                               float* y, void* stream) {
+  TraceRange trace_("mq_linear_container");
   g_last_error.clear();
   mq_status st = check_linear("mq_linear_container", x, M, K, q, alpha, zero, N, r, y);
   if (st != MQ_OK) return st;
@@ -225,6 +232,7 @@ static mq_status check_ovf(const char* who, const uint8_t* q, int64_t N, int64_t
 
 mq_status mq_ep_overflow_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32_t* row_ptr,
                               void* stream) {
+  TraceRange trace_("mq_ep_overflow_rows");
   g_last_error.clear();
   mq_status st = check_ovf("mq_ep_overflow_rows", q, N, K, r);
   if (st != MQ_OK) return st;
@@ -236,6 +244,7 @@ mq_status mq_ep_overflow_rows(const uint8_t* q, int64_t N, int64_t K, int r, int
 
 mq_status mq_ep_overflow_cols(const uint8_t* q, int64_t N, int64_t K, int r, const int32_t* row_ptr,
                               uint16_t* cols, void* stream) {
+  TraceRange trace_("mq_ep_overflow_cols");
   g_last_error.clear();
   mq_status st = check_ovf("mq_ep_overflow_cols", q, N, K, r);
   if (st != MQ_OK) return st;
@@ -249,6 +258,7 @@ mq_status mq_ep_overflow_cols(const uint8_t* q, int64_t N, int64_t K, int r, con
 mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed, const float* alpha,
                        const float* zero, int64_t N, int r, const int32_t* row_ptr,
                        const uint16_t* cols, float* y, void* stream) {
+  TraceRange trace_("mq_linear_ep");
   g_last_error.clear();
   mq_status st = check_linear("mq_linear_ep", x, M, K, packed, alpha, zero, N, r, y);
   if (st != MQ_OK) return st;
@@ -271,6 +281,7 @@ size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
 mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
                            int64_t Dkv, int64_t F, int64_t head_dim, float* h, void* scratch,
                            size_t scratch_bytes, int flags, void* stream) {
+  TraceRange trace_("mq_chain_forward");
   g_last_error.clear();
   const char* who = "mq_chain_forward";
   if (!layers || !h || !scratch) return fail(MQ_ERR_INVALID_ARG, "%s: null pointer", who);
@@ -305,6 +316,7 @@ mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M
 
 mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, int n_lins,
                            const int* widths, int n_layers, int64_t M, void* stream) {
+  TraceRange trace_("mq_stack_forward");
   g_last_error.clear();
   if (!lins || !layer_of_lin || !widths) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: null host array");
   if (n_lins < 1 || n_layers < 1) return fail(MQ_ERR_INVALID_ARG, "mq_stack_forward: need n_lins >= 1 and n_layers >= 1");
@@ -331,6 +343,7 @@ mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, 
 }
 
 mq_status mq_device_status(void* stream) {
+  TraceRange trace_("mq_device_status");
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");

@@ -125,11 +125,12 @@ __device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo
 // two 16-bit halves at once (h2 = 2^(s-1) in both halves, kmask the code's
 // bits in both halves after the shift by s).
 template <int R>
-__device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p1, uint32_t (&v)[16],
-                                         uint32_t h2 = 0, uint32_t kmask = 0, int sh = 0) {
+__device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, const uint8_t* p1,
+                                         uint32_t (&v)[16], uint32_t h2 = 0, uint32_t kmask = 0,
+                                         int sh = 0) {
   if constexpr (R == 10 || R == 11) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
-    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0b);
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -171,7 +172,7 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p1, u
     }
   } else {  // R == 8: bytes, 4 codes per word
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
-    const uint4 b = *reinterpret_cast<const uint4*>(p0 + 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(p0b);
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 16; ++j)
@@ -319,11 +320,27 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       // plane 0 rows hold 64 codes (8*b0 bytes); this warp's 32 codes are half
       // of them. Plane 1 rows hold a 16-byte chunk: 64 codes at b1 = 2, 128 at
       // b1 = 1 (of which this stage uses the half it % 2).
-      const uint8_t* r0 = st + p.off_p0 + row * (8 * b0) + h * (4 * b0);
+      // plane-0 rows of 32 bytes (b0 = 4) and 64 bytes (b0 = 8) are stored in
+      // 32- and 64-byte swizzled atoms: 16-byte chunk c of row `row` sits at
+      // chunk c ^ ((row / 4) % 2), resp. c ^ ((row / 2) % 4)
+      const uint8_t* p0row = st + p.off_p0 + row * (8 * b0);
+      const uint8_t* r0;
+      const uint8_t* r0b;
+      if constexpr (b0 == 8) {
+        const int x = (row >> 1) & 3;
+        r0 = p0row + 16 * ((2 * h) ^ x);
+        r0b = p0row + 16 * ((2 * h + 1) ^ x);
+      } else if constexpr (b0 == 4) {
+        r0 = p0row + 16 * (h ^ ((row >> 2) & 1));
+        r0b = r0;
+      } else {
+        r0 = p0row + h * (4 * b0);
+        r0b = r0;
+      }
       const uint8_t* r1 = st + p.off_p1 + row * 16 +
                           (b1 == 1 ? (it % 2) * 8 + h * 4 : h * 8);
       uint32_t v[16];
-      decode32<R>(r0, r1, v, ch2, ckm, cs);
+      decode32<R>(r0, r0b, r1, v, ch2, ckm, cs);
       tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();
@@ -406,10 +423,12 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   if (job.ep_rows) return cudaErrorNotSupported;  // Extra Precision lists serve the decode path only
 
   static thread_local GemmParams gp;
-  cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, true);
+  cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, 128);
   if (e != cudaSuccess) return e;
+  // plane-0 rows of 32 or 64 bytes arrive swizzled, so that the decode
+  // threads (one weight row each) read them without bank conflicts
   e = encode_map_2d(&gp.map_p0, job.packed, uint64_t(job.N), uint64_t(job.K) * b0 / 8,
-                    8u * b0, kBN, 1);
+                    8u * b0, kBN, 1, b0 == 8 ? 64 : b0 == 4 ? 32 : 0);
   if (e != cudaSuccess) return e;
   if (b1) {
     e = encode_map_2d(&gp.map_p1, job.packed + job.N * job.K * b0 / 8, uint64_t(job.N),

@@ -896,7 +896,7 @@ cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
   // 128-byte plane-0 rows go with 256-row units and the 128-byte swizzle
   const uint32_t rows = P0 == 128 ? 256u : 128u;
   cudaError_t e = encode_map_2d(&out2[0], j.packed, uint64_t(j.N), uint64_t(j.K) * b0 / 8,
-                                static_cast<uint32_t>(P0), rows, 1, P0 == 128);
+                                static_cast<uint32_t>(P0), rows, 1, P0 == 128 ? 128 : 0);
   if (e != cudaSuccess || !b1) return e;
   return encode_map_2d(&out2[1], j.packed + j.N * j.K * b0 / 8, uint64_t(j.N),
                        uint64_t(j.K) * b1 / 8, static_cast<uint32_t>(P0 / 2), rows, 1);

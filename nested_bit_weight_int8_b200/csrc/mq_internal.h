@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdint>
 #include <vector>
 
@@ -90,12 +92,14 @@ void set_last_error(const char* msg);
 
 // 2-D tensor map over a row-major matrix of `rows` x `row_elems` elements of
 // `elem_bytes` bytes (1: uint8, 2: bf16), box `box_inner` x `box_rows`,
-// out-of-bounds elements read as zero, no swizzle unless `swizzle128` (then
-// the box rows are stored in 128-byte swizzled atoms; box_inner * elem_bytes
-// must be 128). Cached per arguments.
+// out-of-bounds elements read as zero. `swizzle_bytes` 0 stores the box
+// plainly; 32, 64 or 128 stores its rows in swizzled atoms of that span
+// (box_inner * elem_bytes must equal it; the 16-byte chunk c of row r then sits
+// at chunk c ^ ((r / (128 / span)) % (span / 16)) and the destination must be
+// aligned to 8 rows of the span). Cached per arguments.
 cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t row_elems,
                           uint32_t box_inner, uint32_t box_rows, int elem_bytes,
-                          bool swizzle128 = false);
+                          int swizzle_bytes = 0);
 int sm_count();
 
 // gamma, beta: per-row clipping factors of Eq. 3, or null for Eq. 1.
@@ -146,5 +150,14 @@ void release_chain_graphs();
 // Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
 // cudaErrorNotSupported for shapes it does not serve (nothing launched).
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);
+
+// An NVTX range around every entry point that launches work, so a timeline
+// tool shows each library call (without a tool attached it costs a branch).
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
 
 }  // namespace mq

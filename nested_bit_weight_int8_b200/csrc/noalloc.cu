@@ -69,6 +69,7 @@ using namespace mq;
 extern "C" mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, const void* packed,
                                        const float* alpha, const float* zero, int64_t N, int r,
                                        float* y, void* stream) {
+  mq::TraceRange trace_("mq_linear_noalloc");
   set_last_error("");
   if (!x || !packed || !alpha || !zero || !y) return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: null pointer");
   if (r != 8 && r != 6 && r != 4 && r != 3 && r != 2)

@@ -17,7 +17,7 @@ namespace {
 
 std::mutex g_tm_mutex;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t, uint32_t, int, bool>, CUtensorMap> g_maps;
+std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t, uint32_t, int, int>, CUtensorMap> g_maps;
 
 cudaError_t load_encoder() {
   if (g_encode) return cudaSuccess;
@@ -33,9 +33,11 @@ cudaError_t load_encoder() {
 }  // namespace
 
 cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t row_elems,
-                          uint32_t box_inner, uint32_t box_rows, int elem_bytes, bool swizzle128) {
+                          uint32_t box_inner, uint32_t box_rows, int elem_bytes, int swizzle_bytes) {
+  if (swizzle_bytes != 0 && swizzle_bytes != 32 && swizzle_bytes != 64 && swizzle_bytes != 128)
+    return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lk(g_tm_mutex);
-  auto key = std::make_tuple(base, rows, row_elems, box_inner, box_rows, elem_bytes, swizzle128);
+  auto key = std::make_tuple(base, rows, row_elems, box_inner, box_rows, elem_bytes, swizzle_bytes);
   auto it = g_maps.find(key);
   if (it != g_maps.end()) {
     *out = it->second;
@@ -52,7 +54,10 @@ cudaError_t encode_map_2d(CUtensorMap* out, const void* base, uint64_t rows, uin
       elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUresult r = g_encode(&m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                        : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (g_maps.size() > 4096) g_maps.clear();
