@@ -22,6 +22,10 @@
  *    this build does not serve); mq_last_error() then describes it.
  *  - A CUDA launch failure returns MQ_ERR_CUDA. A bounded device-side wait
  *    that gave up is reported by mq_device_status() as MQ_ERR_TIMEOUT.
+ *  - A library built with MQ_DEBUG_BOUNDS (libmq_debug.so) checks its device
+ *    indices (activation layout, shared-memory reads, Extra Precision
+ *    columns); a failed check skips the access and mq_device_status()
+ *    reports MQ_ERR_BOUNDS. The normal build compiles the checks out.
  *  - No C++ exception crosses this interface.
  *  - The library keeps a small per-(device, stream) workspace of device
  *    memory for its own scratch (activation copies, row sums, error word).
@@ -50,7 +54,8 @@ typedef enum mq_status {
   MQ_ERR_INVALID_ARG = 1,
   MQ_ERR_UNSUPPORTED = 2,
   MQ_ERR_CUDA = 3,
-  MQ_ERR_TIMEOUT = 4
+  MQ_ERR_TIMEOUT = 4,
+  MQ_ERR_BOUNDS = 5
 } mq_status;
 
 typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1 } mq_dtype;

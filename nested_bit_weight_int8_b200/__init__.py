@@ -15,7 +15,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmq.so")
+# MQ_LIBRARY=debug loads the build with device index checks (libmq_debug.so).
+LIB_PATH = os.path.join(_HERE, "libmq_debug.so" if os.environ.get("MQ_LIBRARY") == "debug"
+                        else "libmq.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -23,7 +25,7 @@ if not os.path.exists(LIB_PATH):
         "(nvcc, sm_100a). There is no fallback implementation.")
 _lib = ctypes.CDLL(LIB_PATH)
 
-MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CUDA, MQ_ERR_TIMEOUT = range(5)
+MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CUDA, MQ_ERR_TIMEOUT, MQ_ERR_BOUNDS = range(6)
 MQ_F32, MQ_BF16 = 0, 1
 WIDTHS = (8, 6, 4, 3, 2)
 

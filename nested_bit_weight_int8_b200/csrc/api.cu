@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/mq.h"
+#include "mq_device.cuh"
 #include "mq_internal.h"
 
 namespace mq {
@@ -356,6 +357,8 @@ mq_status mq_device_status(void* stream) {
   if (v != 0) {
     e = cudaMemset(err, 0, sizeof(uint32_t));
     if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+    if (v & kErrBounds)
+      return fail(MQ_ERR_BOUNDS, "a device index check failed (flags 0x%x); its outputs are undefined", v);
     return fail(MQ_ERR_TIMEOUT, "a kernel gave up a bounded wait (flags 0x%x); its outputs are undefined", v);
   }
   return MQ_OK;

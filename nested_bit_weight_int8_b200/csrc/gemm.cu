@@ -339,8 +339,11 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       }
       const uint8_t* r1 = st + p.off_p1 + row * 16 +
                           (b1 == 1 ? (it % 2) * 8 + h * 4 : h * 8);
-      uint32_t v[16];
-      decode32<R>(r0, r0b, r1, v, ch2, ckm, cs);
+      uint32_t v[16] = {};
+      const uint8_t* st_end = st + p.stage_bytes;
+      // (r1 is read only by widths with a second plane)
+      if (MQ_IN_BOUNDS(r0 + 16 <= st_end && r0b + 16 <= st_end && (b1 == 0 || r1 + 8 <= st_end), p.err))
+        decode32<R>(r0, r0b, r1, v, ch2, ckm, cs);
       tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();

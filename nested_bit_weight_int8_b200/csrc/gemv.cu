@@ -300,7 +300,8 @@ __device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses
 template <int R, int NT, int TW, int Q>
 __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, const Cdec& cd, float (&ch)[TW][NT][2][4]) {
+                                           int gbase, const Cdec& cd, uint32_t* errp,
+                                           float (&ch)[TW][NT][2][4]) {
   uint4 xb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -309,7 +310,9 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
     // mbarrier wait before the unit is a memory barrier it cannot cross
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t a = xaddr[nt] + static_cast<uint32_t>(gbase + Q) * xstep[nt];
-    xb[nt] = *reinterpret_cast<const uint4*>(smem + a);
+    xb[nt] = make_uint4(0u, 0u, 0u, 0u);
+    if (MQ_IN_BOUNDS(a + 16u <= dynamic_smem_bytes(), errp))
+      xb[nt] = *reinterpret_cast<const uint4*>(smem + a);
   }
   // two operand planes for r = 3, 6 (low/high bit planes)
   constexpr int NPL = (Geo<R>::b1 != 0) ? 2 : 1;
@@ -338,9 +341,10 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
 template <int R, int NT, int TW, int... Qs>
 __device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, const Cdec& cd, float (&ch)[TW][NT][2][4],
+                                           int gbase, const Cdec& cd, uint32_t* errp,
+                                           float (&ch)[TW][NT][2][4],
                                            std::integer_sequence<int, Qs...>) {
-  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, cd, ch), ...);
+  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, cd, errp, ch), ...);
 }
 
 // One staged unit for this warp's 16-row tiles. All sub-steps are unrolled
@@ -354,7 +358,8 @@ template <int R, int NT>
 __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* st1,
                                              const uint32_t (&xaddr)[NT],
                                              const uint32_t (&xstep)[NT], int warp, int lane,
-                                             const Cdec& cd, float (&ch)[Tiling<NT>::TW][NT][2][4]) {
+                                             const Cdec& cd, uint32_t* errp,
+                                             float (&ch)[Tiling<NT>::TW][NT][2][4]) {
   using G = Geo<R>;
   using TL = Tiling<NT>;
   constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0, P1 = TL::P0 / 2;
@@ -383,7 +388,7 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
   }
 #pragma unroll
   for (int s = 0; s < NSUB; ++s)
-    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, cd, ch,
+    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, cd, errp, ch,
                           std::make_integer_sequence<int, G::W8>{});
 }
 
@@ -507,7 +512,7 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
 #pragma unroll
           for (int j = 0; j < 4; ++j) { ch[T][b][0][j] = 0.f; ch[T][b][1][j] = 0.f; }
       // the plane pitches and rows follow from the batch tiles (Tiling)
-      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, cd, ch);
+      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, cd, p.err, ch);
 #pragma unroll
       for (int T = 0; T < TW; ++T)
 #pragma unroll
@@ -709,6 +714,7 @@ struct PrepEp {
 constexpr int kMaxEpJobs = 8;
 template <int CAP>
 struct PrepParams {
+  uint32_t* err;  // device error word (index checks of the debug build)
   int M, n_layout, n_sum, n_zero, n_ep;
   int rows;  // weight rows per unit: the height of a zeroed row block
   PrepLayout lay[CAP];
@@ -786,7 +792,8 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       const int t = rem / L.w8, q = rem % L.w8;
       const int64_t off = int64_t(kc) * M * L.kc * 2 +
                           ((int64_t(s * L.w8 + q) * M + m) * 4 + t) * 16;
-      *reinterpret_cast<uint4*>(L.xf + off) = v;
+      if (MQ_IN_BOUNDS(off + 16 <= int64_t(L.n_kc) * M * L.kc * 2, p.err))
+        *reinterpret_cast<uint4*>(L.xf + off) = v;
     }
   }
   // (4) Extra Precision sums: one warp per (job, row). With M' the next power
@@ -810,7 +817,10 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       if (m < M) {
         const __nv_bfloat16* xr = E.x + int64_t(m) * E.K;
 #pragma unroll 4
-        for (int j = beg + jo; j < end; j += P) acc += __bfloat162float(xr[E.cols[j]]);
+        for (int j = beg + jo; j < end; j += P) {
+          const int k = E.cols[j];
+          if (MQ_IN_BOUNDS(k < E.K, p.err)) acc += __bfloat162float(xr[k]);
+        }
       }
       for (int o = mp; o < 32; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (jo == 0 && m < M) E.out[int64_t(m) * E.N + n] = acc;
@@ -1127,7 +1137,15 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   }
 
   // Prep launch.
+  uint32_t* err = nullptr;
+  if (fixed) {
+    err = fixed->err;
+  } else {
+    e = get_error_word(&err);
+    if (e != cudaSuccess) return e;
+  }
   pp.M = M;
+  pp.err = err;
   pp.n_layout = n_layouts;
   pp.n_sum = n_sums;
   pp.n_zero = n_zero;
@@ -1156,13 +1174,6 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.off_x = off_x;
   gp.pitch0 = P0;
   gp.pitch1 = P1;
-  uint32_t* err = nullptr;
-  if (fixed) {
-    err = fixed->err;
-  } else {
-    e = get_error_word(&err);
-    if (e != cudaSuccess) return e;
-  }
   gp.err = err;
   gp.wait_ns = wait_limit_ns();
 

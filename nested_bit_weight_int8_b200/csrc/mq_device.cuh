@@ -13,6 +13,23 @@ constexpr uint32_t kErrWaitFull = 1u;      // consumer waited too long for data
 constexpr uint32_t kErrWaitEmpty = 2u;     // producer waited too long for a free stage
 constexpr uint32_t kErrDrain = 4u;         // copies still in flight at exit
 constexpr uint32_t kErrMma = 8u;           // tensor-core pipeline wait gave up
+constexpr uint32_t kErrBounds = 16u;       // a debug build's index check failed
+
+// Index checks of the debug build (compiled with MQ_DEBUG_BOUNDS): a check
+// that fails sets kErrBounds in the error word and the guarded access is
+// skipped, so a bad index becomes a status instead of a fault. In the normal
+// build the checks compile to nothing.
+#ifdef MQ_DEBUG_BOUNDS
+#define MQ_IN_BOUNDS(cond, errp) ((cond) ? true : (atomicOr((errp), ::mq::kErrBounds), false))
+#else
+#define MQ_IN_BOUNDS(cond, errp) true
+#endif
+
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t v;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

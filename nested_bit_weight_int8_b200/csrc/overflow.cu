@@ -14,6 +14,7 @@
 
 #include <cstdint>
 
+#include "mq_device.cuh"
 #include "mq_internal.h"
 
 namespace mq {
@@ -95,12 +96,13 @@ __global__ void __launch_bounds__(kScanThreads) ovf_scan_kernel(int32_t* __restr
 // cols[row_ptr[n] ..] = the positions of row n, increasing.
 __global__ void __launch_bounds__(kOvfThreads)
 ovf_fill_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K, uint32_t thr4,
-                const int32_t* __restrict__ row_ptr, uint16_t* __restrict__ cols) {
+                const int32_t* __restrict__ row_ptr, uint16_t* __restrict__ cols, uint32_t* err) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = int64_t(gridDim.x) * (kOvfThreads / 32);
   for (int64_t n = int64_t(blockIdx.x) * (kOvfThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
     const uint8_t* row = q + n * K;
     int base = row_ptr[n];
+    const int row_end = row_ptr[n + 1];
     for (int64_t k0 = 0; k0 < K; k0 += 32 * 16) {
       const int64_t k = k0 + int64_t(lane) * 16;
       uint32_t m = 0;
@@ -115,7 +117,8 @@ ovf_fill_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K, uint32_t th
       int pos = base + incl - cnt;
       while (m) {
         const int bit = __ffs(m) - 1;
-        cols[pos++] = static_cast<uint16_t>(k + bit);
+        if (MQ_IN_BOUNDS(pos < row_end, err)) cols[pos] = static_cast<uint16_t>(k + bit);
+        ++pos;
         m &= m - 1;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
@@ -147,7 +150,10 @@ cudaError_t launch_ovf_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32
 
 cudaError_t launch_ovf_cols(const uint8_t* q, int64_t N, int64_t K, int r, const int32_t* row_ptr,
                             uint16_t* cols, cudaStream_t stream, int sms) {
-  ovf_fill_kernel<<<ovf_grid(N, sms), kOvfThreads, 0, stream>>>(q, N, K, threshold4(r), row_ptr, cols);
+  uint32_t* err = nullptr;
+  cudaError_t e = get_error_word(&err);
+  if (e != cudaSuccess) return e;
+  ovf_fill_kernel<<<ovf_grid(N, sms), kOvfThreads, 0, stream>>>(q, N, K, threshold4(r), row_ptr, cols, err);
   return cudaGetLastError();
 }
 

@@ -136,3 +136,16 @@ def test_ep_entry_points_reject():
     assert mq.raw_status("mq_linear_ep", *ok, 2, None, F, F, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.raw_status("mq_linear_ep", *ok, 2, F, F + 1, F, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.raw_status("mq_linear_ep", F, 33, 256, F, F, F, 64, 2, F, F, F, None) == mq.MQ_ERR_UNSUPPORTED
+
+
+def test_debug_build_exports_the_same_entry_points():
+    # the build with device index checks (libmq_debug.so) is a drop-in
+    # replacement: same header, same exported names
+    import ctypes
+    import os
+    path = os.path.join(os.path.dirname(mq.LIB_PATH), "libmq_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libmq_debug.so not built")
+    lib = ctypes.CDLL(path)
+    for name in mq.EXPORTED:
+        assert hasattr(lib, name), name
