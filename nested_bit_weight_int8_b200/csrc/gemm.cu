@@ -341,6 +341,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
                           (b1 == 1 ? (it % 2) * 8 + h * 4 : h * 8);
       uint32_t v[16] = {};
       const uint8_t* st_end = st + p.stage_bytes;
+      (void)st_end;  // read only by the debug build's checks
       // (r1 is read only by widths with a second plane)
       if (MQ_IN_BOUNDS(r0 + 16 <= st_end && r0b + 16 <= st_end && (b1 == 0 || r1 + 8 <= st_end), p.err))
         decode32<R>(r0, r0b, r1, v, ch2, ckm, cs);
