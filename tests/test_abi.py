@@ -149,3 +149,50 @@ def test_debug_build_exports_the_same_entry_points():
     lib = ctypes.CDLL(path)
     for name in mq.EXPORTED:
         assert hasattr(lib, name), name
+
+
+def test_quantize_clipped_rejects():
+    F = FAKE
+    ok = (F, 1, 4, 64)
+    assert mq.raw_status("mq_quantize_int8_clipped", *ok, None, F, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8_clipped", *ok, F, None, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8_clipped", *ok, F + 2, F, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8_clipped", F, 7, 4, 64, F, F, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.raw_status("mq_quantize_int8_clipped", F, 1, 0, 64, F, F, F, F, F, None) == mq.MQ_ERR_INVALID_ARG
+
+
+def test_chain_rejects_on_the_host():
+    # every argument error is caught before anything launches (no GPU needed)
+    import ctypes
+    F = FAKE
+    layer = mq.ChainLayer()
+    layer.r = 4
+    for i in range(5):
+        layer.packed[i] = F
+        layer.alpha[i] = F
+        layer.zero[i] = F
+    arr = (mq.ChainLayer * 1)(layer)
+    need = mq.chain_scratch_bytes(1, 512, 128, 1024)
+    assert need > 0
+    base = (arr, 1, 1, 512, 128, 1024, 64, F, F, need, 0, None)
+
+    def call(**kw):
+        a = list(base)
+        names = ["layers", "n", "M", "D", "Dkv", "F", "hd", "h", "scratch", "bytes", "flags", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return mq._chain(*a)
+
+    assert call(n=0) == mq.MQ_ERR_INVALID_ARG
+    assert call(M=0) == mq.MQ_ERR_INVALID_ARG
+    assert call(M=33) == mq.MQ_ERR_INVALID_ARG
+    assert call(D=500) == mq.MQ_ERR_INVALID_ARG
+    assert call(hd=48) == mq.MQ_ERR_INVALID_ARG           # does not divide Dkv
+    assert call(bytes=need - 1) == mq.MQ_ERR_INVALID_ARG
+    assert call(scratch=F + 128) == mq.MQ_ERR_INVALID_ARG  # not 256-byte aligned
+    assert call(flags=4) == mq.MQ_ERR_INVALID_ARG
+    assert call(h=None) == mq.MQ_ERR_INVALID_ARG
+    layer_bad = (mq.ChainLayer * 1)(layer)
+    layer_bad[0].r = 5
+    assert call(layers=layer_bad) == mq.MQ_ERR_INVALID_ARG
+    assert mq.last_error()
