@@ -177,17 +177,9 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t m
 // bf16x2 powers of two 2^e in both halves (OR-ing a code into the mantissa
 // gives 2^e + code * 2^(e-7+p) exactly).
 constexpr uint32_t kMag4 = 0x40804080u, kMag8 = 0x41004100u, kMag16 = 0x41804180u,
-                   kMag32 = 0x42004200u, kMag64 = 0x42804280u, kMag128 = 0x43004300u,
+                   kMag32 = 0x42004200u, kMag64 = 0x42804280u,
                    kMag256 = 0x43804380u;
-constexpr uint32_t kMaskP3b2 = 0x00180018u, kMaskP5b2 = 0x00600060u, kMaskP3b4 = 0x00780078u,
-                   kMaskP0b4 = 0x000F000Fu;
-
-// bf16x2 a - b, exact here: both are small integers (magic + code, magic).
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
+constexpr uint32_t kMaskP3b2 = 0x00180018u, kMaskP5b2 = 0x00600060u, kMaskP3b4 = 0x00780078u;
 
 // Two bytes of w (chosen by the byte_perm selectors, which put the byte under
 // the exponent of 2^23) as an exact bf16x2 pair of integers 0..255.
@@ -200,21 +192,19 @@ __device__ __forceinline__ uint32_t bytes_bf16x2(uint32_t w, uint32_t sel_lo, ui
 }
 
 // The pair of 2-bit codes at half-word position P (0, 2, ..., 14) of a plane
-// word as bf16x2. Positions 0-4 need no shift, 6-10 one shift by 6, 12-14 one
-// by 12, so a word costs two shifts and eight LOP3s. The code lands at bit
-// p = P mod 6 of each half, under the magic 2^(7-p) that gives it weight 1:
-// offsets 32 (p = 2) and 8 (p = 4) stay, and the 128 of p = 0 is subtracted
-// again at once on the FMA pipe, which keeps the fp32 sums small.
+// word as bf16x2. A left shift by 1 puts positions 0-4 at bits 1, 3, 5 of
+// each half, right shifts by 5 and 11 do the same for 6-10 and 12-14, so a
+// word costs three shifts and eight LOP3s. The code sits under the magic
+// 2^(7-p) that gives it weight 1: offsets 64, 16, 4 (the bits shifted in
+// from the other half fall outside the mask). An earlier form used shifts of
+// 0, 6, 12 and took the offset 128 of bit 0 out with a bf16x2 subtract: one
+// instruction more per word.
 template <int P>
 __device__ __forceinline__ uint32_t pick2(uint32_t w) {
-  constexpr int sh = P <= 4 ? 0 : (P <= 10 ? 6 : 12);
+  constexpr int sh = P <= 4 ? -1 : (P <= 10 ? 5 : 11);
   constexpr int p = P - sh;
   constexpr uint32_t mask = 0x00030003u << p;
-  if constexpr (p == 0) {
-    return bf16x2_sub(and_or(w >> sh, mask, kMag128), kMag128);
-  } else {
-    return and_or(w >> sh, mask, p == 2 ? kMag32 : kMag8);
-  }
+  return and_or(shift_to<sh>(w), mask, p == 1 ? kMag64 : p == 3 ? kMag16 : kMag4);
 }
 
 // Decoded A registers of one MMA for one weight row: x0 fills k-slots
@@ -284,7 +274,7 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
 // stay small next to the code unit (at most 32 at r = 2), so the fp32 sums
 // lose little to cancellation when the offsets are taken out again.
 __device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses]) {
-  constexpr float r2[kClasses] = {0.f, 32.f, 8.f, 0.f, 32.f, 8.f, 0.f, 32.f};
+  constexpr float r2[kClasses] = {64.f, 16.f, 4.f, 64.f, 16.f, 4.f, 64.f, 16.f};
   constexpr float r3[4] = {80.f, 36.f, 32.f, 12.f};
   constexpr float r6[4] = {272.f, 80.f, 272.f, 80.f};
   // the container sliced on load: one magic for every class
@@ -952,12 +942,12 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
 // always holds the same plane bytes per row (two planes hold 1.5x), while the
 // decode and MMA work grows with the codes in it: per-unit times of
 // single-width stacks on B200 at M = 1 put r = 4 at about 1.26x and r = 2 at
-// about 1.93x an r = 8 unit; r = 3 and 6 are scaled from their planes.
+// about 1.88x an r = 8 unit; r = 3 and 6 are scaled from their planes.
 int64_t unit_cost(const LinearJob& j) {
   switch (decode_kind(j)) {
     case 8: return 100;
     case 4: return 126;
-    case 2: return 193;
+    case 2: return 188;
     case 6: return 183;
     case 10: case 11: return 110;  // one 8-bit plane, one MMA per 16 codes, more decode work
     default: return 301;  // 3

@@ -103,6 +103,7 @@ ovf_fill_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K, uint32_t th
     const uint8_t* row = q + n * K;
     int base = row_ptr[n];
     const int row_end = row_ptr[n + 1];
+    (void)row_end;  // read only by the debug build's checks
     for (int64_t k0 = 0; k0 < K; k0 += 32 * 16) {
       const int64_t k = k0 + int64_t(lane) * 16;
       uint32_t m = 0;
