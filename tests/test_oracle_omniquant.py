@@ -65,3 +65,15 @@ def test_pins_catch_an_unclipped_range():
     w = np.array([[-2.0, -1.0, 0.0, 0.5078125, 1.5, 2.984375, 5.96875, -0.0078125]])
     q, a, z = oracle.quantize_omniquant(w, np.array([1.0]), np.array([0.5]))
     assert q[0].tolist() != [0, 0, 64, 96, 160, 255, 255, 64]
+
+
+def test_synthetic_extra_bucket_recipe():
+    # the Extra Precision workload: about 2.5% of each row's container values
+    # fall in the int2 extra bucket (Eq. 8 code above the Eq. 6 code), as the
+    # errata section reports for trained models
+    w = synth.f32_from_bf16_bits(synth.extra_bucket_weights(64, 4096, 11)).astype(np.float64)
+    q, _, _ = oracle.quantize_minmax(w)
+    frac = (oracle.slice_codes(q, 2, clamp=False) != oracle.slice_codes(q, 2)).mean()
+    assert 0.02 < frac < 0.035
+    # each row's range is pinned, so its extremes map to 0 and 255
+    assert (q.min(axis=1) == 0).all() and (q.max(axis=1) == 255).all()
