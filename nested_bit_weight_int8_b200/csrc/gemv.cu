@@ -23,14 +23,14 @@
 // Exactness of the operands. A code c (0 <= c < 2^b, b <= 4) is OR-ed into
 // the mantissa of a bf16 power of two 2^e at a bit position p, which yields
 // exactly 2^e + c * 2^(e-7+p); choosing p and e so that the code weight is 1
-// (or 4, 16 for the high plane of r = 3, 6; 16 for the high nibble of r = 8)
-// gives the integer value off + weight*c, exact in bf16. The offsets "off"
+// (or 4, 16 for the high plane of r = 3, 6) gives the integer value
+// off + weight*c, exact in bf16. A byte (r = 8) has one significant bit too
+// many for this; it goes through fp32 instead (below). The offsets "off"
 // sum to O_m = sum_k x[m,k] off(k), which depends only on k mod 16 and is
 // removed in the epilogue from per-class activation sums computed once:
 //   y = A_n (acc - O_m) - B_n Sx_m,  A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n.
-// Offsets stay <= 272 (none at r = 8, whose bytes go through fp32 exactly),
-// so fp32 partial sums stay small (accuracy), and two codes are decoded per
-// shift+LOP3 pair (issue budget at r = 2).
+// Offsets stay <= 272 (none at r = 8), so fp32 partial sums stay small
+// (accuracy), and two codes are decoded per LOP3 (issue budget at r = 2).
 //
 // Slicing on load. A linear may also stream the int8 container itself (the
 // r = 8 plane) and slice each byte while decoding, so one stored matrix serves
