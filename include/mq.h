@@ -55,7 +55,8 @@ typedef enum mq_status {
   MQ_ERR_UNSUPPORTED = 2,
   MQ_ERR_CUDA = 3,
   MQ_ERR_TIMEOUT = 4,
-  MQ_ERR_BOUNDS = 5
+  MQ_ERR_BOUNDS = 5,
+  MQ_ERR_IO = 6
 } mq_status;
 
 typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1 } mq_dtype;
@@ -268,6 +269,22 @@ MQ_API size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t 
 MQ_API mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
                                   int64_t Dkv, int64_t F, int64_t head_dim, float* h,
                                   void* scratch, size_t scratch_bytes, int flags, void* stream);
+
+/*
+ * The int8 container as a file: the one stored artifact, from which every
+ * width is sliced. Host buffers (the caller copies device data). Layout,
+ * little-endian: "MQC8", version 1 (uint32), N, K (int64), q (N x K uint8,
+ * row-major), alpha, zero (N fp32 each), then the CRC-32 (IEEE, reflected) of
+ * everything before it. Errors: MQ_ERR_INVALID_ARG for null pointers, sizes
+ * below 1, or a file of another shape (load); MQ_ERR_IO for a file that
+ * cannot be opened, written or read, is truncated, has trailing bytes, is not
+ * a container of this version, or fails its checksum.
+ */
+MQ_API mq_status mq_container_save(const char* path, const uint8_t* q, const float* alpha,
+                                   const float* zero, int64_t N, int64_t K);
+MQ_API mq_status mq_container_info(const char* path, int64_t* N, int64_t* K);
+MQ_API mq_status mq_container_load(const char* path, uint8_t* q, float* alpha, float* zero,
+                                   int64_t N, int64_t K);
 
 /* Bytes of the device array that mq_linear_noalloc works in (1.25 MiB). */
 #define MQ_NOALLOC_SCRATCH_BYTES (1280u * 1024u)

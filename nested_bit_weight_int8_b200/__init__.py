@@ -25,7 +25,8 @@ if not os.path.exists(LIB_PATH):
         "(nvcc, sm_100a). There is no fallback implementation.")
 _lib = ctypes.CDLL(LIB_PATH)
 
-MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CUDA, MQ_ERR_TIMEOUT, MQ_ERR_BOUNDS = range(6)
+(MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CUDA, MQ_ERR_TIMEOUT, MQ_ERR_BOUNDS,
+ MQ_ERR_IO) = range(7)
 MQ_F32, MQ_BF16 = 0, 1
 WIDTHS = (8, 6, 4, 3, 2)
 
@@ -74,6 +75,10 @@ _chain_bytes = _sig("mq_chain_scratch_bytes", ctypes.c_size_t, [_i64, _i64, _i64
 _chain = _sig("mq_chain_forward", _int,
               [ctypes.POINTER(ChainLayer), _int, _i64, _i64, _i64, _i64, _i64, _vp, _vp,
                ctypes.c_size_t, _int, _vp])
+_c_save = _sig("mq_container_save", _int, [ctypes.c_char_p, _vp, _vp, _vp, _i64, _i64])
+_c_info = _sig("mq_container_info", _int,
+               [ctypes.c_char_p, ctypes.POINTER(_i64), ctypes.POINTER(_i64)])
+_c_load = _sig("mq_container_load", _int, [ctypes.c_char_p, _vp, _vp, _vp, _i64, _i64])
 _linear_noalloc = _sig("mq_linear_noalloc", _int,
                       [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp])
 _device_status = _sig("mq_device_status", _int, [_vp])
@@ -85,7 +90,7 @@ EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8"
             "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc",
             "mq_quantize_int8_clipped", "mq_linear_container", "mq_ep_overflow_rows",
             "mq_ep_overflow_cols", "mq_linear_ep", "mq_chain_scratch_bytes",
-            "mq_chain_forward")
+            "mq_chain_forward", "mq_container_save", "mq_container_info", "mq_container_load")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -205,6 +210,35 @@ class ChainPlan:
                       _ptr(scratch), nbytes, MQ_CHAIN_GRAPH if graph else 0, _stream(stream)))
 
 
+def save_container(path: str, q, alpha, zero) -> None:
+    """Writes the int8 container (q N x K uint8, alpha and zero N fp32; torch
+    tensors on any device) to `path` in the library's file format."""
+    qh, ah, zh = (t.detach().contiguous().cpu() for t in (q, alpha, zero))
+    n, k = qh.shape
+    _check(_c_save(os.fsencode(path), qh.data_ptr(), ah.data_ptr(), zh.data_ptr(), n, k))
+
+
+def container_shape(path: str) -> tuple:
+    """(N, K) of a container file."""
+    n, k = _i64(0), _i64(0)
+    _check(_c_info(os.fsencode(path), ctypes.byref(n), ctypes.byref(k)))
+    return n.value, k.value
+
+
+def load_container(path: str, device=None):
+    """Reads a container file into (q, alpha, zero) torch tensors on `device`
+    (the host by default); the checksum is verified."""
+    import torch
+    n, k = container_shape(path)
+    q = torch.empty((n, k), dtype=torch.uint8)
+    a = torch.empty(n, dtype=torch.float32)
+    z = torch.empty(n, dtype=torch.float32)
+    _check(_c_load(os.fsencode(path), q.data_ptr(), a.data_ptr(), z.data_ptr(), n, k))
+    if device is not None:
+        q, a, z = q.to(device), a.to(device), z.to(device)
+    return q, a, z
+
+
 def linear_noalloc(x, M: int, K: int, packed, alpha, zero, N: int, r: int, y, stream=None) -> None:
     """As linear() for 1 <= M <= 32, but working in the library's fixed device
     array instead of allocating a workspace (for callers that cannot allocate).
@@ -261,4 +295,5 @@ def raw_status(fn_name: str, *args) -> int:
             "mq_quantize_int8_clipped": _quantize_clipped,
             "mq_linear": _linear, "mq_linear_noalloc": _linear_noalloc,
             "mq_linear_container": _linear_container, "mq_linear_ep": _linear_ep,
-            "mq_ep_overflow_rows": _ovf_rows, "mq_ep_overflow_cols": _ovf_cols}[fn_name](*args)
+            "mq_ep_overflow_rows": _ovf_rows, "mq_ep_overflow_cols": _ovf_cols,
+            "mq_container_save": _c_save, "mq_container_load": _c_load}[fn_name](*args)

@@ -17,6 +17,15 @@
 #include "mq_internal.h"
 
 namespace mq {
+
+// The container file (container_io.cu); nonzero return = failure with `why`
+// (2: a file of another shape).
+int container_save(const char* path, const uint8_t* q, const float* alpha, const float* zero, int64_t N,
+                   int64_t K, char* why, size_t why_len);
+int container_info(const char* path, int64_t* N, int64_t* K, char* why, size_t why_len);
+int container_load(const char* path, uint8_t* q, float* alpha, float* zero, int64_t N, int64_t K, char* why,
+                   size_t why_len);
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -312,6 +321,37 @@ mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M
                             static_cast<int>(F), static_cast<int>(head_dim), h, scratch,
                             (flags & MQ_CHAIN_GRAPH) != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, who);
+  return MQ_OK;
+}
+
+mq_status mq_container_save(const char* path, const uint8_t* q, const float* alpha, const float* zero,
+                            int64_t N, int64_t K) {
+  TraceRange trace_("mq_container_save");
+  g_last_error.clear();
+  if (!path || !q || !alpha || !zero) return fail(MQ_ERR_INVALID_ARG, "mq_container_save: null pointer");
+  if (N < 1 || K < 1) return fail(MQ_ERR_INVALID_ARG, "mq_container_save: N and K must be >= 1");
+  char why[512];
+  if (container_save(path, q, alpha, zero, N, K, why, sizeof(why)) != 0) return fail(MQ_ERR_IO, "%s", why);
+  return MQ_OK;
+}
+
+mq_status mq_container_info(const char* path, int64_t* N, int64_t* K) {
+  g_last_error.clear();
+  if (!path || !N || !K) return fail(MQ_ERR_INVALID_ARG, "mq_container_info: null pointer");
+  char why[512];
+  if (container_info(path, N, K, why, sizeof(why)) != 0) return fail(MQ_ERR_IO, "%s", why);
+  return MQ_OK;
+}
+
+mq_status mq_container_load(const char* path, uint8_t* q, float* alpha, float* zero, int64_t N, int64_t K) {
+  TraceRange trace_("mq_container_load");
+  g_last_error.clear();
+  if (!path || !q || !alpha || !zero) return fail(MQ_ERR_INVALID_ARG, "mq_container_load: null pointer");
+  if (N < 1 || K < 1) return fail(MQ_ERR_INVALID_ARG, "mq_container_load: N and K must be >= 1");
+  char why[512];
+  const int rc = container_load(path, q, alpha, zero, N, K, why, sizeof(why));
+  if (rc == 2) return fail(MQ_ERR_INVALID_ARG, "%s", why);
+  if (rc != 0) return fail(MQ_ERR_IO, "%s", why);
   return MQ_OK;
 }
 
