@@ -196,3 +196,31 @@ def test_chain_rejects_on_the_host():
     layer_bad[0].r = 5
     assert call(layers=layer_bad) == mq.MQ_ERR_INVALID_ARG
     assert mq.last_error()
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 and a C program
+    # links against the library and calls it (host-only calls, no GPU)
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(mq.LIB_PATH)
+    src = tmp_path / "t.c"
+    src.write_text(
+        '#include "mq.h"\n'
+        "int main(void) {\n"
+        "  int64_t n = 0, k = 0;\n"
+        '  if (mq_container_info("/nonexistent/x.mqc", &n, &k) != MQ_ERR_IO) return 1;\n'
+        "  if (mq_packed_bytes(4, 64, 2) != 64) return 2;\n"
+        "  return mq_version() > 0 ? 0 : 3;\n"
+        "}\n")
+    exe = tmp_path / "t"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"), str(src),
+                        "-L", libdir, "-l:" + os.path.basename(mq.LIB_PATH), "-Wl,-rpath," + libdir,
+                        "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
