@@ -97,8 +97,10 @@ quantize_rows_kernel(const T* __restrict__ w, int64_t N, int64_t K, bool vec,
       }
       // Eq. 1: alpha = (max - min) / (2^8 - 1), z = -min / alpha.
       float al = __fdiv_rn(__fsub_rn(b, a), 255.0f);
-      // constant row (or an empty clipped range): alpha = 1, z = -min
-      if (!(al > 0.0f)) al = 1.0f;
+      // constant row (or an empty clipped range): alpha = max(|min| 2^-8,
+      // 2^-126), both exact, so z = -min / alpha is -256 sign(min) (or
+      // min 2^126) and alpha (0 - z) = min exactly
+      if (!(al > 0.0f)) al = fmaxf(fabsf(a) * 0.00390625f, 1.17549435e-38f);
       const float z = __fdiv_rn(-a, al);
       s_alpha = al;
       s_zero = z;

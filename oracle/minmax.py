@@ -17,15 +17,20 @@ double rounding innocuous?", 1995).
 Readings where the pages are silent:
 * round(.) is round-half-to-even (IEEE default);
 * z is kept as a real (float32), not rounded to an integer;
-* a row whose alpha is 0 (max == min) gets alpha = 1, z = -min, so every code
-  is 0 and alpha * (0 - z) = min reproduces the row exactly.
+* a row whose alpha is 0 (max == min) gets alpha = max(|min| 2^-8, 2^-126)
+  (both powers-of-two scalings, exact in float32) and z = -min / alpha
+  (= -256 sign(min), or min 2^126 for |min| < 2^-118): every code is 0 and
+  alpha * (0 - z) = min reproduces the row exactly. Eq. 1 divides by zero
+  there; alpha on the row's own scale (rather than 1) keeps the scaled code
+  sums alpha 2^(8 - r) sum_k x_k c_k of the sliced product small next to the
+  row's values, as they are for every other row.
 """
 from __future__ import annotations
 
 import numpy as np
 
 FP32_CONTRACT = (
-    "d = f32(max - min); alpha = f32(d / (2^c - 1)); alpha == 0 -> alpha = 1; "
+    "d = f32(max - min); alpha = f32(d / (2^c - 1)); alpha == 0 -> alpha = max(|min| 2^-8, 2^-126); "
     "z = f32(-min / alpha); t = f32(f32(w / alpha) + z); q = clamp(rint_even(t), 0, 2^c - 1)"
 )
 
@@ -49,12 +54,18 @@ def quantize_minmax(w: np.ndarray, c: int = 8):
     d = _f32(mx - mn)
     alpha = _f32(d / levels)
     degenerate = alpha == 0.0
-    alpha = np.where(degenerate, 1.0, alpha)
+    alpha = np.where(degenerate, degenerate_alpha(mn), alpha)
     zero = _f32(-mn / alpha)
     with np.errstate(over="ignore", invalid="ignore"):
         t = _f32(_f32(w / alpha[:, None]) + zero[:, None])
     q = np.clip(np.rint(t), 0.0, levels)
     return q.astype(np.uint8), alpha.astype(np.float32), zero.astype(np.float32)
+
+
+def degenerate_alpha(m: np.ndarray) -> np.ndarray:
+    """The scale of a row with no range: max(|m| 2^-8, 2^-126), with m the
+    row's minimum (Eq. 1) or clipped minimum (Eq. 3)."""
+    return np.maximum(np.abs(np.asarray(m, dtype=np.float64)) * 2.0 ** -8, 2.0 ** -126)
 
 
 def dequantize(q: np.ndarray, alpha: np.ndarray, zero: np.ndarray) -> np.ndarray:

@@ -17,12 +17,14 @@ alpha = f32(d / (2^c - 1)), z = f32(-bmin / alpha), t = f32(f32(w / alpha) + z),
 q = clamp(rint_even(t), 0, 2^c - 1).
 
 Reading where the page is silent: a row whose clipped range is empty or
-inverted (alpha <= 0) gets alpha = 1 and z = -bmin, the same rule Eq. 1's
-constant rows follow.
+inverted (alpha <= 0) gets alpha = max(|bmin| 2^-8, 2^-126) and z = -bmin / alpha,
+the rule Eq. 1's constant rows follow with bmin in place of min.
 """
 from __future__ import annotations
 
 import numpy as np
+
+from .minmax import degenerate_alpha
 
 
 def _f32(a):
@@ -48,7 +50,7 @@ def quantize_omniquant(w: np.ndarray, gamma: np.ndarray, beta: np.ndarray, c: in
     bmin = _f32(beta * w.min(axis=1))
     alpha = _f32(_f32(gmax - bmin) / levels)
     empty = alpha <= 0.0
-    alpha = np.where(empty, 1.0, alpha)
+    alpha = np.where(empty, degenerate_alpha(bmin), alpha)
     zero = _f32(-bmin / alpha)
     with np.errstate(over="ignore", invalid="ignore"):
         t = _f32(_f32(w / alpha[:, None]) + zero[:, None])

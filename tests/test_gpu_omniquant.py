@@ -86,7 +86,7 @@ def test_clipped_range_rules():
     w[4] *= 1e4
     gamma = np.array([0.9, 0.5, 0.7, 1.0, 0.8, 0.0, 0.3, 1.0], dtype=np.float32)
     beta = np.array([0.9, 0.5, 1.0, 0.7, 0.8, 0.0, 1.0, 0.3], dtype=np.float32)
-    # row 5: gamma = beta = 0 (empty range, alpha = 1); rows 6, 7 one-sided clipping
+    # row 5: gamma = beta = 0 (empty range, alpha = 2^-126); rows 6, 7 one-sided clipping
     _assert_clipped_equal(w, w.astype(np.float64), "f32", gamma, beta)
     # inverted range: gamma * max < beta * min for an all-positive row
     w2 = (np.abs(rng.standard_normal((2, 64))) + 2.0).astype(np.float32)

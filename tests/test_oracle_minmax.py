@@ -39,13 +39,18 @@ def test_closed_form_quarter_scale():
 
 
 def test_degenerate_row():
-    w = np.full((2, 64), 0.375)
+    w = np.full((4, 64), 0.375)
     w[1] = -2.5
+    w[2] = 0.0
+    w[3] = -2.0 ** -130
     q, a, z = oracle.quantize_minmax(w)
     assert np.all(q == 0)
-    assert np.all(a == 1.0)
-    assert z[0] == -0.375 and z[1] == 2.5
+    # alpha = |min| / 256 (the row's own scale), 2^-126 at the bottom of the range
+    assert a.tolist() == [0.375 / 256, 2.5 / 256, 2.0 ** -126, 2.0 ** -126]
+    assert z.tolist() == [-256.0, 256.0, 0.0, 2.0 ** -4]
     assert np.array_equal(oracle.dequantize(q, a, z), w)
+    for r in (8, 6, 4, 3, 2):
+        assert np.array_equal(oracle.dequant_slice(q, a, z, r), w)
 
 
 @pytest.mark.parametrize("law", ["gauss", "t"])

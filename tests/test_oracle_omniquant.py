@@ -56,8 +56,18 @@ def test_invariants_inside_and_outside_the_clipped_range(seed):
 def test_empty_range_rule():
     w = np.array([[0.4, -1.6, 2.5, 3.49]])
     q, a, z = oracle.quantize_omniquant(w, np.array([0.0]), np.array([0.0]))
-    assert a[0] == 1.0 and z[0] == 0.0
-    assert q[0].tolist() == [0, 0, 2, 3]   # clamp(round_half_even(w)), 2.5 -> 2
+    # bmin = 0: alpha = 2^-126, z = 0, so every weight saturates by its sign
+    assert a[0] == np.float32(2.0 ** -126) and z[0] == 0.0
+    assert q[0].tolist() == [255, 0, 255, 255]
+    # an all-negative row with gamma = 0 still has a range: gmax = 0, bmin < 0
+    wn = np.array([[-1.0, -2.0, -3.0, -0.5]])
+    q, a, z = oracle.quantize_omniquant(wn, np.array([0.0]), np.array([0.5]))
+    # gmax = 0 * (-0.5) = -0, bmin = 0.5 * -3 = -1.5: range [-1.5, 0] is valid
+    assert a[0] == np.float32(1.5 / 255)
+    q, a, z = oracle.quantize_omniquant(-wn, np.array([0.0]), np.array([1.0]))
+    # all-positive row, gamma = 0: gmax = 0 < bmin = 0.5, inverted
+    assert a[0] == np.float32(0.5 / 256) and z[0] == -256.0
+    assert q[0].tolist() == [255, 255, 255, 0]   # w / alpha - 256: 0.5 -> 0
 
 
 def test_pins_catch_an_unclipped_range():
