@@ -34,7 +34,7 @@ constexpr int kGlueThreads = 256;
 constexpr float kEps = 1e-6f;
 
 // One CTA per batch row: v = h + add (add may be null), written to h_out if
-// given; xn = bf16(v / sqrt(mean(v^2) + eps)).
+// given; xn = bf16(v / sqrt(mean(v^2) + eps)) if xn is given.
 __global__ void __launch_bounds__(kGlueThreads)
 rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ add, float* __restrict__ h_out,
                __nv_bfloat16* __restrict__ xn, int D) {
@@ -51,6 +51,7 @@ rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ add, float
     if (h_out) h_out[int64_t(m) * D + k] = v;
     ss = fmaf(v, v, ss);
   }
+  if (!xn) return;  // the last layer's residual add alone
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((tid & 31) == 0) red[tid >> 5] = ss;
@@ -197,9 +198,11 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
     if (e != cudaSuccess) return e;
     LinearJob jd = job(4, bf(L.act), D, F, fp(L.dn));
     if ((e = run_gemv_fixed_n(&jd, 1, M, s, fx)) != cudaSuccess) return e;
-    // h = h1 + down, and the next layer's normalized input
+    // h = h1 + down, and the next layer's normalized input (none after the
+    // last layer, whose intermediates then all stay in the scratch)
+    __nv_bfloat16* next_xn = l + 1 < c.n_layers ? bf(L.xn) : nullptr;
     e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(fp(L.h1)),
-                   static_cast<const float*>(fp(L.dn)), c.h, bf(L.xn), D);
+                   static_cast<const float*>(fp(L.dn)), c.h, next_xn, D);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -213,6 +216,12 @@ std::map<std::vector<uint64_t>, cudaGraphExec_t> g_graphs;
 
 size_t chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
   return chain_layout(M, D, Dkv, F).total;
+}
+
+void chain_views(int64_t M, int64_t D, int64_t Dkv, int64_t F, size_t out[10]) {
+  const ChainLayout L = chain_layout(M, D, Dkv, F);
+  const size_t v[10] = {L.xn, L.qkv, L.a, L.o, L.h1, L.xn1, L.g, L.u, L.act, L.dn};
+  for (int i = 0; i < 10; ++i) out[i] = v[i];
 }
 
 cudaError_t run_chain(const mq_chain_layer* layers, int n_layers, int M, int D, int Dkv, int F, int hd,

@@ -58,19 +58,44 @@ def silu(g: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g))
 
 
+U32 = 2.0 ** -24  # unit roundoff of fp32 (round to nearest)
+
+
+def bf16_flip(v: np.ndarray, e: np.ndarray) -> np.ndarray:
+    """Largest change of bf16(v') over all v' with |v' - v| <= e: rounding to
+    nearest is monotone, so it is reached at v - e or v + e (0 where no
+    rounding boundary lies within e of v)."""
+    r = to_bf16(v)
+    return np.maximum(np.abs(to_bf16(v + e) - r), np.abs(to_bf16(v - e) - r))
+
+
+def rmsnorm_f32_error(h: np.ndarray, eps: float = 1e-6, threads: int = 256) -> np.ndarray:
+    """Bound on |v32 - rmsnorm(h)| for an fp32 RMSNorm of the same fp32 input
+    h whose sum of squares is formed by `threads` threads of D / threads
+    sequential fused multiply-adds and a reduction tree of depth 16: that sum
+    is off by at most (D / threads + 16) u relatively (u = 2^-24); the mean,
+    square root, reciprocal and the scaling add 4 u, all relative to |v|."""
+    d = h.shape[1]
+    gamma = (d / threads + 16) * U32
+    return np.abs(rmsnorm(h, eps)) * (gamma / 2 + 4 * U32)
+
+
+def swiglu_f32_error(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """Bound on |a32 - silu(g) u| for fp32 evaluation of g / (1 + exp(-g)) * u
+    on the same fp32 g, u: exp within 2 ulp, the add, the division and the
+    product within half an ulp each: 8 u relative."""
+    return 8 * U32 * np.abs(silu(g) * u)
+
+
 def chain_forward(h: np.ndarray, layers, d: int, dkv: int, head_dim: int, eps: float = 1e-6,
-                  trace: list | None = None, bound: list | None = None) -> np.ndarray:
+                  trace: list | None = None) -> np.ndarray:
     """Runs the layers in order on the residual stream h (M x d).
 
     layers: list of dicts with float64 weight matrices "qkv" ((d + 2 dkv) x d),
     "o" (d x d), "gate" and "up" (f x d), "down" (d x f). If `trace` is a
-    list, the residual stream after each layer is appended to it. If `bound`
-    is a list, the running sum over the layers so far of the two residual
-    linears' element-wise bounds 1e-3 (|a| |W_o|^T + |act| |W_down|^T) (the
-    per-linear accuracy bound of the decode path) is appended after each layer.
+    list, the residual stream after each layer is appended to it.
     """
     h = np.asarray(h, dtype=np.float64).copy()
-    acc = np.zeros_like(h)
     for L in layers:
         xn = to_bf16(rmsnorm(h, eps))
         qkv = xn @ L["qkv"].T
@@ -81,7 +106,4 @@ def chain_forward(h: np.ndarray, layers, d: int, dkv: int, head_dim: int, eps: f
         h = h1 + act @ L["down"].T
         if trace is not None:
             trace.append(h.copy())
-        if bound is not None:
-            acc = acc + 1e-3 * (np.abs(a) @ np.abs(L["o"]).T + np.abs(act) @ np.abs(L["down"]).T)
-            bound.append(acc.copy())
     return h

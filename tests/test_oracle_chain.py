@@ -102,23 +102,51 @@ def test_pins_catch_a_dropped_residual():
     assert not np.array_equal(no_residual(h, [_zero_layer(d, dkv, f)]), h)
 
 
-def test_chain_bound_accumulates_the_residual_linears():
-    # one layer: the bound is 1e-3 (|a| |Wo|^T + |act| |Wdown|^T), and zero
-    # weights give a zero bound
-    d, dkv, f, hd = 16, 8, 32, 4
-    rng = np.random.default_rng(5)
-    h = rng.standard_normal((2, d))
-    b = []
-    ch.chain_forward(h, [_zero_layer(d, dkv, f)] * 2, d, dkv, hd, bound=b)
-    assert len(b) == 2 and not b[0].any() and not b[1].any()
-    L = {k: rng.standard_normal(v.shape) for k, v in _zero_layer(d, dkv, f).items()}
-    b = []
-    ch.chain_forward(h, [L, L], d, dkv, hd, bound=b)
-    xn = ch.to_bf16(ch.rmsnorm(h))
-    a = ch.to_bf16(ch.attention_single_token(xn @ L["qkv"].T, d, dkv, hd))
-    h1 = h + a @ L["o"].T
-    xn1 = ch.to_bf16(ch.rmsnorm(h1))
-    act = ch.to_bf16(ch.silu(xn1 @ L["gate"].T) * (xn1 @ L["up"].T))
-    want = 1e-3 * (np.abs(a) @ np.abs(L["o"]).T + np.abs(act) @ np.abs(L["down"]).T)
-    assert np.allclose(b[0], want, rtol=1e-12)
-    assert np.all(b[1] > b[0])
+def test_bf16_flip_hand_values():
+    v = np.array([1.0, 1.0 + 2.0 ** -8 - 2.0 ** -12, 1.0 + 2.0 ** -9, -3.0, -3.0])
+    e = np.array([0.0, 2.0 ** -11, 2.0 ** -12, 2.0 ** -7, 2.0 ** -7 + 2.0 ** -10])
+    # exact value stays; just below a tie the error reaches it (one bf16 step
+    # 2^-7 at 1); mid-interval with a small error nothing moves; -3 -+ 2^-7 are
+    # ties that round back to -3 (even); a little further they reach the
+    # neighbours -3 -+ 2^-6
+    assert ch.bf16_flip(v, e).tolist() == [0.0, 2.0 ** -7, 0.0, 0.0, 2.0 ** -6]
+
+
+def _rmsnorm_like_the_gpu(h32: np.ndarray, threads: int = 256) -> np.ndarray:
+    """fp32 RMSNorm with the reduction structure the bound assumes: each of
+    `threads` threads sums every threads-th square sequentially with fp32
+    fused multiply-adds, then a tree adds the partial sums."""
+    d = h32.shape[1]
+    out = np.empty_like(h32)
+    for i, row in enumerate(h32):
+        part = np.zeros(threads, dtype=np.float32)
+        for k in range(0, d, threads):
+            blk = row[k:k + threads]
+            part[:len(blk)] = (part[:len(blk)].astype(np.float64) + blk.astype(np.float64) ** 2).astype(np.float32)
+        while len(part) > 1:
+            part = (part[0::2] + part[1::2]).astype(np.float32)
+        inv = np.float32(1.0) / np.sqrt(np.float32(part[0] / np.float32(d)) + np.float32(1e-6))
+        out[i] = row * inv
+    return out.astype(np.float64)
+
+
+@pytest.mark.parametrize("scale", [1e-3, 1.0, 1e3])
+def test_rmsnorm_f32_bound_covers_an_fp32_rmsnorm(scale):
+    rng = np.random.default_rng(int(scale * 7) + 1)
+    h = (rng.standard_normal((4, 4096)) * scale).astype(np.float32)
+    v32 = _rmsnorm_like_the_gpu(h)
+    v64 = ch.rmsnorm(h.astype(np.float64))
+    err = np.abs(v32 - v64)
+    bound = ch.rmsnorm_f32_error(h.astype(np.float64))
+    assert np.all(err <= bound)
+    # and it is not vacuous: the observed worst case reaches a visible part of it
+    assert (err / bound).max() > 0.01
+
+
+def test_swiglu_f32_bound_covers_fp32_evaluation():
+    rng = np.random.default_rng(3)
+    g = (rng.standard_normal(100000) * 4).astype(np.float32)
+    u = rng.standard_normal(100000).astype(np.float32)
+    a32 = (g / (np.float32(1.0) + np.exp(-g)) * u).astype(np.float64)
+    g64, u64 = g.astype(np.float64), u.astype(np.float64)
+    assert np.all(np.abs(a32 - ch.silu(g64) * u64) <= ch.swiglu_f32_error(g64, u64))
