@@ -160,11 +160,8 @@ class Stack:
         layers = len(self.widths)
         mats = synth.WORKLOADS[WORKLOAD]["mats"]
         self.Ks = sorted({k for _, _, k in mats})
-        gen = torch.Generator(device=dev)
-        self.x = {}
-        for k in self.Ks:
-            gen.manual_seed(2000 + M + k)
-            self.x[k] = torch.randn((M, k), generator=gen, device=dev).to(torch.bfloat16)
+        self.x = {k: synth.device_activations(M, k, 2000 + M + k, dev) for k in self.Ks}
+        self.seed_base = seed_base
         self.lins, self.lol, self.bytes_by_width, self.layer_of = [], [], {}, []
         self.packed_bytes = 0
         self.rows_total = 0
@@ -175,8 +172,7 @@ class Stack:
         for layer in range(layers):
             r = self.widths[layer]
             for j, (_, n, k) in enumerate(mats):
-                gen.manual_seed(seed_base + 5 * layer + j)
-                w = (torch.randn((n, k), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+                w = synth.device_gaussian_weights(n, k, seed_base + 5 * layer + j, dev)
                 q = torch.empty((n, k), dtype=torch.uint8, device=dev)
                 a = torch.empty(n, dtype=torch.float32, device=dev)
                 z = torch.empty(n, dtype=torch.float32, device=dev)

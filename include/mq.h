@@ -91,7 +91,8 @@ MQ_API size_t mq_packed_bytes(int64_t N, int64_t K, int r);
  * Arithmetic contract (IEEE binary32, each operation correctly rounded, no
  * contraction): d = max - min; alpha = d / 255; z = -min / alpha;
  * t = (w / alpha) + z; q = clamp(round-half-to-even(t), 0, 255). A row whose
- * alpha rounds to 0 (max == min) gets alpha = 1 and z = -min (all codes 0).
+ * alpha rounds to 0 (max == min) gets alpha = max(|min| 2^-8, 2^-126) and
+ * z = -min / alpha (exact: all codes 0 and alpha (0 - z) = min).
  *   w     : N x K, fp32 (dtype MQ_F32) or bf16 (MQ_BF16), 4-byte aligned.
  *   q     : N x K uint8 out.   alpha, zero : N fp32 out.
  * Requires N >= 1, K >= 1; weights finite with a finite range.
@@ -108,7 +109,8 @@ MQ_API mq_status mq_quantize_int8(const void* w, int dtype, int64_t N, int64_t K
  * so weights outside [beta_n min, gamma_n max] saturate at 0 or 255. Same
  * arithmetic contract as mq_quantize_int8, with gmax = gamma * max and
  * bmin = beta * min rounded first; a row whose clipped range is empty or
- * inverted (alpha <= 0) gets alpha = 1 and z = -bmin. gamma = beta = 1 gives
+ * inverted (alpha <= 0) gets alpha = max(|bmin| 2^-8, 2^-126) and
+ * z = -bmin / alpha. gamma = beta = 1 gives
  * exactly mq_quantize_int8.
  *   gamma, beta : N fp32 (device), 4-byte aligned, finite (OmniQuant keeps
  *                 them in (0, 1)). Other arguments as mq_quantize_int8.
@@ -266,6 +268,29 @@ typedef struct mq_chain_layer {
 } mq_chain_layer;
 #define MQ_CHAIN_GRAPH 1
 MQ_API size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F);
+
+/*
+ * Where mq_chain_forward leaves the intermediate values of its LAST layer
+ * inside the caller's scratch: byte offsets from the scratch pointer, valid
+ * once the call's stream has completed, for inspecting a token's step (and
+ * for checking each step against a reference on the chain's own inputs).
+ * Every buffer is row-major with M rows:
+ *   xn   M x D bf16           bf16(rmsnorm(h_in)), the input of qkv
+ *   qkv  M x (D + 2 Dkv) fp32
+ *   a    M x D bf16           the attention output, the input of o
+ *   o    M x D fp32           a Wo^T
+ *   h1   M x D fp32           h_in + o (fp32 add)
+ *   xn1  M x D bf16           bf16(rmsnorm(h1))
+ *   g, u M x F fp32           gate and up products
+ *   act  M x F bf16           bf16(silu(g) u)
+ *   down M x D fp32           act Wdown^T; h_out = h1 + down (fp32 add)
+ * Returns MQ_ERR_INVALID_ARG for sizes mq_chain_scratch_bytes rejects.
+ */
+typedef struct mq_chain_views {
+  size_t xn, qkv, a, o, h1, xn1, g, u, act, down;
+} mq_chain_views;
+MQ_API mq_status mq_chain_scratch_views(int64_t M, int64_t D, int64_t Dkv, int64_t F,
+                                        mq_chain_views* out);
 MQ_API mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
                                   int64_t Dkv, int64_t F, int64_t head_dim, float* h,
                                   void* scratch, size_t scratch_bytes, int flags, void* stream);
@@ -305,8 +330,10 @@ MQ_API mq_status mq_container_load(const char* path, uint8_t* q, float* alpha, f
  * MQ_NOALLOC_SCRATCH_BYTES. The first 256 bytes hold a wait-error word; the
  * rest holds the fragment-ordered activation blocks and activation sums.
  * Every GPU that loads the library holds this array until the process exits.
- * It is enough for M * K up to 524288 (e.g. M = 32 with K = 16384). A call
- * that needs more returns MQ_ERR_INVALID_ARG with the sizes in
+ * It is enough for M * K up to 524288 (e.g. M = 32 with K = 16384), except
+ * at M = 1 with r = 8, 4 or 2, whose inputs are staged as seven integer
+ * digits (7.1 to 7.5 bytes each): there K up to 174592, 180480 and 183808.
+ * A call that needs more returns MQ_ERR_INVALID_ARG with the sizes in
  * mq_last_error() and launches nothing.
  *
  * Arguments, layouts and accuracy: as mq_linear, with 1 <= M <= 32.
@@ -320,8 +347,9 @@ MQ_API mq_status mq_container_load(const char* path, uint8_t* q, float* alpha, f
  * call wrote. Each call rewrites on the device all the scratch it reads, and
  * zeroes y there before accumulating. Calls whose kernels overlap on the GPU race: two streams,
  * or two host threads on one device. Serialize them. A bounded wait that gave
- * up leaves y undefined. It is recorded in the array's error word, not in the
- * word that mq_device_status() reads.
+ * up leaves y undefined and is recorded in the array's error word;
+ * mq_device_status() reads and clears that word too (as MQ_ERR_TIMEOUT) and
+ * allocates nothing, so such a caller can check its calls with it.
  */
 MQ_API mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, const void* packed,
                                    const float* alpha, const float* zero, int64_t N, int r,
@@ -330,8 +358,10 @@ MQ_API mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, const vo
 /*
  * Synchronizes `stream`, then reports whether any kernel launched by this
  * library on the current device gave up a bounded wait (MQ_ERR_TIMEOUT; the
- * outputs of that call are then undefined) and clears the flag.
- * Returns MQ_ERR_CUDA if the synchronization itself failed.
+ * outputs of that call are then undefined) and clears the flag. It reads the
+ * error word of the per-device workspace and that of mq_linear_noalloc's
+ * fixed array, and allocates nothing. Returns MQ_ERR_CUDA if the
+ * synchronization itself failed.
  */
 MQ_API mq_status mq_device_status(void* stream);
 

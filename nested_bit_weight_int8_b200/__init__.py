@@ -72,6 +72,13 @@ _ovf_cols = _sig("mq_ep_overflow_cols", _int, [_vp, _i64, _i64, _int, _vp, _vp, 
 _linear_ep = _sig("mq_linear_ep", _int,
                   [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _vp])
 _chain_bytes = _sig("mq_chain_scratch_bytes", ctypes.c_size_t, [_i64, _i64, _i64, _i64])
+
+
+class ChainViews(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("xn", "qkv", "a", "o", "h1", "xn1", "g", "u", "act", "down")]
+
+
+_chain_views = _sig("mq_chain_scratch_views", _int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ChainViews)])
 _chain = _sig("mq_chain_forward", _int,
               [ctypes.POINTER(ChainLayer), _int, _i64, _i64, _i64, _i64, _i64, _vp, _vp,
                ctypes.c_size_t, _int, _vp])
@@ -90,7 +97,8 @@ EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8"
             "mq_release_workspace", "mq_debug_set_wait_limit_ns", "mq_linear_noalloc",
             "mq_quantize_int8_clipped", "mq_linear_container", "mq_ep_overflow_rows",
             "mq_ep_overflow_cols", "mq_linear_ep", "mq_chain_scratch_bytes",
-            "mq_chain_forward", "mq_container_save", "mq_container_info", "mq_container_load")
+            "mq_chain_forward", "mq_container_save", "mq_container_info", "mq_container_load",
+            "mq_chain_scratch_views")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -185,6 +193,13 @@ def linear_ep(x, M: int, K: int, packed, alpha, zero, N: int, r: int, row_ptr, c
 
 def chain_scratch_bytes(M: int, D: int, Dkv: int, F: int) -> int:
     return int(_chain_bytes(M, D, Dkv, F))
+
+
+def chain_scratch_views(M: int, D: int, Dkv: int, F: int) -> dict:
+    """Byte offsets of the last layer's intermediates in the chain's scratch."""
+    v = ChainViews()
+    _check(_chain_views(M, D, Dkv, F, ctypes.byref(v)))
+    return {n: int(getattr(v, n)) for n, _ in ChainViews._fields_}
 
 
 class ChainPlan:

@@ -110,6 +110,14 @@ cudaError_t get_error_word(uint32_t** out) {
   return cudaSuccess;
 }
 
+uint32_t* find_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lk(g_ws_mutex);
+  auto it = g_error_words.find(dev);
+  return it == g_error_words.end() ? nullptr : it->second;
+}
+
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 
 void set_last_error(const char* msg) { g_last_error = msg; }
@@ -288,6 +296,16 @@ size_t mq_chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
   return chain_scratch_bytes(M, D, Dkv, F);
 }
 
+mq_status mq_chain_scratch_views(int64_t M, int64_t D, int64_t Dkv, int64_t F, mq_chain_views* out) {
+  g_last_error.clear();
+  if (!out) return fail(MQ_ERR_INVALID_ARG, "mq_chain_scratch_views: null out");
+  if (mq_chain_scratch_bytes(M, D, Dkv, F) == 0) return fail(MQ_ERR_INVALID_ARG, "mq_chain_scratch_views: bad sizes");
+  size_t v[10];
+  chain_views(M, D, Dkv, F, v);
+  *out = mq_chain_views{v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], v[8], v[9]};
+  return MQ_OK;
+}
+
 mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M, int64_t D,
                            int64_t Dkv, int64_t F, int64_t head_dim, float* h, void* scratch,
                            size_t scratch_bytes, int flags, void* stream) {
@@ -388,15 +406,24 @@ mq_status mq_device_status(void* stream) {
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
-  uint32_t* err = nullptr;
-  e = get_error_word(&err);
-  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+  // The device's error word exists once any allocating call ran here; this
+  // call does not create it, so a caller of mq_linear_noalloc alone still
+  // allocates nothing.
   uint32_t v = 0;
-  e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
-  if (v != 0) {
-    e = cudaMemset(err, 0, sizeof(uint32_t));
+  if (uint32_t* err = find_error_word()) {
+    e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+    if (v != 0) {
+      e = cudaMemset(err, 0, sizeof(uint32_t));
+      if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+    }
+  }
+  // mq_linear_noalloc's kernels flag a give-up in its fixed array instead
+  uint32_t vn = 0;
+  e = noalloc_take_error(&vn);
+  if (e != cudaSuccess) return cuda_fail(e, "mq_device_status");
+  v |= vn;
+  if (v != 0) {
     if (v & kErrBounds)
       return fail(MQ_ERR_BOUNDS, "a device index check failed (flags 0x%x); its outputs are undefined", v);
     return fail(MQ_ERR_TIMEOUT, "a kernel gave up a bounded wait (flags 0x%x); its outputs are undefined", v);

@@ -14,11 +14,27 @@
 // kernel zeroes exactly those shared row blocks first.
 //
 // CTA = 8 consumer warps + 1 producer warp. The producer stages each unit in
-// shared memory with 1-D bulk copies (cp.async.bulk, one per row and plane)
-// plus one copy of the activation block, signalling an mbarrier. Each
-// consumer warp owns one tile of 16 rows and runs mma.sync m16n8k16 (bf16 in,
-// fp32 accumulate) with the weights as the A operand and the batch (M <= 32,
-// n8 tiles) as B.
+// shared memory with one 2-D TMA box per plane (cp.async.bulk.tensor; rows
+// past N and bytes past K read as zero) plus one bulk copy of the unit's
+// activation block, signalling an mbarrier. Up to 8 batch rows each consumer
+// warp owns two 16-row tiles (128-byte plane rows in the 128-byte swizzle,
+// 256-row units); above 8 it owns one tile (64-byte rows, 128-row units). It
+// runs mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the weights as the A
+// operand and the batch (n8 tiles) as B.
+//
+// One batch row at r = 8, 4, 2 runs on the integer tensor cores instead
+// (mma.sync m16n8k32, u8 x s8 -> s32): the codes are the A operand as plain
+// bytes, with no offset, so r = 8 needs no decode at all, r = 4 one shift and
+// two ANDs per 8 codes, r = 2 three shifts and four ANDs per 16 codes, and one
+// instruction covers 512 weights. A bf16 input is not an integer, so the prep
+// kernel writes each input of a unit exactly as an integer X = x 2^sigma of up
+// to 49 bits, sigma = 48 - E from the unit's largest exponent E, in seven
+// signed 7-bit digits, digit g in batch column g of the MMA (columns free at
+// one batch row). Accumulation is exact in int32; the epilogue weighs column
+// g by 2^(7g - sigma) when it folds the unit. Inputs more than 41 octaves
+// below the unit's largest (or non-finite ones, or a scale outside the fp32
+// range) mark the unit for the bf16 path instead, so the product is exact for
+// every input up to fp32 rounding.
 //
 // Exactness of the operands. A code c (0 <= c < 2^b, b <= 4) is OR-ed into
 // the mantissa of a bf16 power of two 2^e at a bit position p, which yields
@@ -66,6 +82,23 @@ constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header 
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
 constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
 
+// Decode kinds of the planes at one batch row on the integer tensor cores:
+// kDkI8 + r for r = 8, 4, 2. A unit is 256 rows x 128 plane bytes (1024 / r
+// codes). Its staged activation block is a 64-byte header (int mode: 0 digits,
+// 1 bf16 fragments; int E, the unit's largest exponent; float O, the offset
+// sum of a bf16 unit) and then slot (s, jj, t, g) of 16 bytes at
+// 64 + (((s * J / 2 + jj) * 4 + t) * kI8Digits + g) * 16, J = 16 / r MMAs per
+// 16-byte chunk: digit g of the 16 inputs of MMAs 2 jj and 2 jj + 1 of chunk
+// 4s + t, in their k-slot order (b0, b1 of each). A mode-1 unit holds the
+// width's bf16 fragments there instead.
+constexpr int kDkI8 = 20;
+constexpr int kI8Digits = 7;
+constexpr int kI8Header = 64;
+__host__ __device__ constexpr uint32_t i8_unit_bytes(int r) {
+  return kI8Header + 2u * static_cast<uint32_t>(16 / r / 2) * 4u * kI8Digits * 16u;  // 960, 1856, 3648
+}
+__host__ __device__ constexpr bool is_i8(int dk) { return dk == kDkI8 + 8 || dk == kDkI8 + 4 || dk == kDkI8 + 2; }
+
 // Geometry of a launch with NT batch tiles of 8. Up to 8 batch rows, each
 // consumer warp owns two 16-row tiles (four independent MMA chains; one
 // activation fragment load feeds two MMAs) over 128-byte plane rows staged in
@@ -95,7 +128,9 @@ struct LinDesc {
   const uint8_t* xf;   // activations in fragment order, n_kc blocks of M*KC bf16
   const float* psum;   // [M][8] activation sums per class (k >> 1) & 7
   int N, K, r, kc, n_kc, unit_begin;
-  int dk;  // decode kind: r for planes, 10 / 11 for the container sliced by Eq. 6 / Eq. 8
+  int dk;  // decode kind: r for planes, 10 / 11 for the container sliced by Eq. 6 / Eq. 8,
+           // kDkI8 + r for the planes on the integer tensor cores
+  uint32_t xunit;  // bytes of one unit's staged activation block
   // Extra Precision on the planes (or null): epc[m * N + n] is the sum of
   // x[m, k] over row n's positions whose Eq. 8 code is one step above the
   // Eq. 6 code, computed by the prep kernel.
@@ -155,7 +190,8 @@ __device__ __forceinline__ Cdec make_cdec(int dk, int r) {
 }
 
 __device__ __forceinline__ void plane_widths_dev(int r, int& b0, int& b1) {
-  b0 = (r == 8 || r >= 10) ? 8 : (r == 4 || r == 6) ? 4 : 2;  // 10, 11: the container
+  // 10, 11: the container; kDkI8 + r: planes of width r
+  b0 = (r == 8 || r == 10 || r == 11 || r == kDkI8 + 8) ? 8 : (r == 4 || r == 6 || r == kDkI8 + 4) ? 4 : 2;
   b1 = (r == 3) ? 1 : (r == 6) ? 2 : 0;
 }
 
@@ -281,7 +317,8 @@ __device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses
   const float cont = static_cast<float>(1 << (dk == 10 ? r : r + 1));
 #pragma unroll
   for (int i = 0; i < kClasses; ++i) {
-    c[i] = dk >= 10 ? cont : r == 8 ? 0.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
+    // the integer kinds take each unit's offsets out when they fold it
+    c[i] = is_i8(dk) ? 0.f : dk >= 10 ? cont : r == 8 ? 0.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
   }
 }
 
@@ -386,7 +423,7 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
 struct Cursor {
   int l, rb, kc;          // linear, row block, k-chunk of the current unit
   int nrb, n_kc, r, N;    // of linear l
-  int dk;                 // its decode kind (width, or 10 / 11 for the container)
+  int dk;                 // its decode kind (width, 10 / 11 for the container, or kDkI8 + r)
 };
 
 template <int RPU, int CAP>
@@ -517,6 +554,159 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
   return true;
 }
 
+// The A registers of MMA j of a 16-byte chunk for one weight row (words
+// w[0..3] of the chunk) on the integer path: codes as bytes, in k-slot order
+// k 4t + i (a0) and 16 + 4t + i (a2).
+//  r = 8: the bytes themselves; a0 = word 2j, a2 = word 2j + 1.
+//  r = 4: word j holds codes u at bit 16 (u % 2) + 4 (u / 2); w & 0x0F0F0F0F
+//         gives codes 0, 4, 1, 5 and (w >> 4) & 0x0F0F0F0F codes 2, 6, 3, 7.
+//  r = 2: word j / 2 holds 16 codes at bit 16 (u % 2) + 2 (u / 2);
+//         (w >> 2i) & 0x03030303 gives codes 2i, 2i + 8, 2i + 1, 2i + 9, and
+//         MMA j takes i = 2 (j % 2) (a0) and i = 2 (j % 2) + 1 (a2).
+template <int R, int J>
+__device__ __forceinline__ void i8_regs(const uint32_t (&w)[4], uint32_t& a0, uint32_t& a2) {
+  if constexpr (R == 8) {
+    a0 = w[2 * J];
+    a2 = w[2 * J + 1];
+  } else if constexpr (R == 4) {
+    a0 = w[J] & 0x0F0F0F0Fu;
+    a2 = (w[J] >> 4) & 0x0F0F0F0Fu;
+  } else {
+    a0 = (w[J / 2] >> (4 * (J % 2))) & 0x03030303u;
+    a2 = (w[J / 2] >> (4 * (J % 2) + 2)) & 0x03030303u;
+  }
+}
+
+// One staged unit at width R on the integer path (one batch row, Tiling<1>):
+// the planes are loaded as for the bf16 path (128-byte swizzle); per chunk
+// J = 16 / R MMAs of 16 rows x 32 k, the digits of MMAs 2jj, 2jj + 1 in one
+// 16-byte load at xaddr + (s * J / 2 + jj) * xstep. MMA j accumulates into
+// chain j % 2.
+template <int R, int... Js>
+__device__ __forceinline__ void i8_chunk(const uint32_t (&lo)[2][2][4], const uint8_t* smem_base,
+                                         uint32_t xaddr, uint32_t xstep, int s, uint32_t* errp,
+                                         int (&ch)[2][2][4], std::integer_sequence<int, Js...>) {
+  // the chunk's digit loads first, then its MMAs
+  uint4 xbs[16 / R / 2];
+#pragma unroll
+  for (int jj = 0; jj < 16 / R / 2; ++jj) {
+    const uint32_t a = xaddr + static_cast<uint32_t>(s * (16 / R / 2) + jj) * xstep;
+    xbs[jj] = make_uint4(0u, 0u, 0u, 0u);
+    if (MQ_IN_BOUNDS(a + 16u <= dynamic_smem_bytes(), errp)) xbs[jj] = *reinterpret_cast<const uint4*>(smem_base + a);
+  }
+  auto mma_j = [&](auto jc) {
+    constexpr int J = decltype(jc)::value;
+    const uint4& xb = xbs[J / 2];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+      uint32_t a0, a1, a2, a3;
+      i8_regs<R, J>(lo[T][0], a0, a2);
+      i8_regs<R, J>(lo[T][1], a1, a3);
+      mma_u8s8_16832(ch[T][J % 2], a0, a1, a2, a3, (J % 2) ? xb.z : xb.x, (J % 2) ? xb.w : xb.y);
+    }
+  };
+  (mma_j(std::integral_constant<int, Js>{}), ...);
+}
+
+template <int R>
+__device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xaddr, uint32_t xstep,
+                                                int warp, int lane, uint32_t* errp, int (&ch)[2][2][4]) {
+  using TL = Tiling<1>;
+  constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t lo[NSUB][TW][2][4];
+#pragma unroll
+  for (int s = 0; s < NSUB; ++s) {
+    const int ci = 4 * s + t;
+#pragma unroll
+    for (int T = 0; T < TW; ++T) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = warp * TL::RPW + 16 * T + g + 8 * h;
+        const int cs = ci ^ (row & 7);  // 128-byte swizzle
+        const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * P0 + cs * 16);
+        lo[s][T][h][0] = v.x; lo[s][T][h][1] = v.y; lo[s][T][h][2] = v.z; lo[s][T][h][3] = v.w;
+      }
+    }
+  }
+  extern __shared__ __align__(128) uint8_t smem[];
+#pragma unroll
+  for (int s = 0; s < NSUB; ++s)
+    i8_chunk<R>(lo[s], smem, xaddr, xstep, s, errp, ch, std::make_integer_sequence<int, 16 / R>{});
+}
+
+// run_segment for the integer kinds (one batch row). Each unit's header says
+// whether the prep kernel wrote digits (mode 0) or, for inputs that the
+// digits cannot hold exactly, the bf16 fragments of the width's bf16 path
+// (mode 1). Thread (g, t) of a digit unit holds the int32 sums of columns 2t
+// and 2t + 1, digits 2t and 2t + 1 (column 7 is zero): it weighs them by
+// 2^(7 digit - sigma), sigma = 48 - E. A bf16 unit's offset sum is taken out by
+// thread t = 0. The partials stay in tot[T][0][0] (row g) and tot[T][0][2]
+// (row g + 8) until the row block is flushed.
+template <int R, int CAP>
+__device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const uint8_t* stages,
+                                               uint64_t* full, uint64_t* empty, volatile int* s_abort,
+                                               int seg, int& s, uint32_t& ph, bool active,
+                                               uint32_t zero_addr, int warp, int lane,
+                                               float (&tot)[2][1][4]) {
+  const int g = lane >> 2, t = lane & 3;
+  for (int i = 0; i < seg; ++i) {
+    if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
+      if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
+      return false;
+    }
+    if (active) {
+      const uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+      extern __shared__ __align__(128) uint8_t smem[];
+      const uint8_t* hdr = st + p.off_x;
+      const uint32_t xs = static_cast<uint32_t>(hdr - smem) + kI8Header;  // data, shared offset
+      const int mode = reinterpret_cast<const int*>(hdr)[0];
+      if (mode == 0) {
+        const int E = reinterpret_cast<const int*>(hdr)[1];
+        int ch[2][2][4];
+#pragma unroll
+        for (int T = 0; T < 2; ++T)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) { ch[T][0][j] = 0; ch[T][1][j] = 0; }
+        const bool live = g < kI8Digits;
+        process_unit_i8<R>(st, live ? xs + static_cast<uint32_t>(t * kI8Digits + g) * 16u : zero_addr,
+                           live ? 4u * kI8Digits * 16u : 0u, warp, lane, p.err, ch);
+        // digit 2t weighs 2^(14t + E - 48), digit 2t + 1 2^(14t + 7 + E - 48)
+        const float w0 = __int_as_float((127 + 14 * t + E - 48) << 23);
+        const float w1 = __int_as_float((127 + 14 * t + 7 + E - 48) << 23);
+#pragma unroll
+        for (int T = 0; T < 2; ++T) {
+          tot[T][0][0] = fmaf(static_cast<float>(ch[T][0][0] + ch[T][1][0]), w0,
+                              fmaf(static_cast<float>(ch[T][0][1] + ch[T][1][1]), w1, tot[T][0][0]));
+          tot[T][0][2] = fmaf(static_cast<float>(ch[T][0][2] + ch[T][1][2]), w0,
+                              fmaf(static_cast<float>(ch[T][0][3] + ch[T][1][3]), w1, tot[T][0][2]));
+        }
+      } else {
+        // bf16 fragments of batch row 0 (lanes g = 0), the width's bf16 decode
+        const float O = t == 0 ? reinterpret_cast<const float*>(hdr)[2] : 0.f;
+        float ch[2][1][2][4];
+#pragma unroll
+        for (int T = 0; T < 2; ++T)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) { ch[T][0][0][j] = 0.f; ch[T][0][1][j] = 0.f; }
+        const uint32_t xa[1] = {g == 0 ? xs + static_cast<uint32_t>(t) * 16u : zero_addr};
+        const uint32_t xstep[1] = {g == 0 ? 64u : 0u};
+        process_unit<R, 1>(st, st + Tiling<1>::RPU * Tiling<1>::P0, xa, xstep, warp, lane, Cdec{0u, 0u, 0u},
+                           p.err, ch);
+#pragma unroll
+        for (int T = 0; T < 2; ++T) {
+          tot[T][0][0] += (ch[T][0][0][0] + ch[T][0][1][0]) - O;
+          tot[T][0][2] += (ch[T][0][0][2] + ch[T][0][1][2]) - O;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == p.stages) { s = 0; ph ^= 1u; }
+  }
+  return true;
+}
+
 template <int NT, int CAP>
 __global__ void __launch_bounds__(kGemvThreads, (NT <= 2 ? 2 : 1))
 gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
@@ -568,7 +758,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
         const CUtensorMap* tm = p.map_table ? p.map_table + 2 * cc.l : &p.maps[2 * cc.l];
         const uint32_t box = TL::RPU * (p.pitch0 + (b1 ? p.pitch1 : 0));
-        const uint32_t bytesx = static_cast<uint32_t>(p.M * p.lin[cc.l].kc * 2);
+        const uint32_t bytesx = p.lin[cc.l].xunit;
         // One 2-D box per plane (128 rows x the unit's bytes; rows past N and
         // bytes past K read as zero) plus the unit's activation block.
         mbar_arrive_expect_tx(&full[s], box + bytesx);
@@ -577,7 +767,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       };
       auto issue_x = [&](const Cursor& cc, int s) {
         const LinDesc& L = p.lin[cc.l];
-        const uint32_t bytesx = static_cast<uint32_t>(p.M * L.kc * 2);
+        const uint32_t bytesx = L.xunit;
         uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
         bulk_g2s(st + p.off_x, L.xf + int64_t(cc.kc) * bytesx, bytesx, &full[s]);
       };
@@ -655,10 +845,37 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
       case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
       case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+      // the host plans the integer kinds only for one batch row
+      case kDkI8 + 8:
+        if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
+        else ok = false;
+        break;
+      case kDkI8 + 4:
+        if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
+        else ok = false;
+        break;
+      case kDkI8 + 2:
+        if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
+        else ok = false;
+        break;
       default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
     }
     if (!ok) break;  // outputs are undefined after a give-up; the flag says so
     if (active) {
+      if (is_i8(c.dk)) {
+        // add up the digit partials of the quad: thread t = 0 then holds
+        // batch row 0 of rows g and g + 8, as flush_rows expects
+#pragma unroll
+        for (int T = 0; T < TL::TW; ++T) {
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            float v = tot[T][0][j];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            tot[T][0][j] = v;
+          }
+        }
+      }
 #pragma unroll
       for (int T = 0; T < TL::TW; ++T) flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, T, lane, tot[T]);
     }
@@ -680,6 +897,7 @@ struct PrepLayout {
   uint8_t* xf;
   int K, kc, w8, n_kc;
   int perm02;  // byte planes pair codes (c0, c2), (c1, c3): store x0, x2, x1, x3
+  int i8;      // width r of a digit layout (integer kinds, one batch row), else 0
 };
 struct PrepSum {
   const __nv_bfloat16* x;
@@ -706,6 +924,7 @@ template <int CAP>
 struct PrepParams {
   uint32_t* err;  // device error word (index checks of the debug build)
   int M, n_layout, n_sum, n_zero, n_ep;
+  int n_i8;  // units of all digit layouts (phase 2b)
   int rows;  // weight rows per unit: the height of a zeroed row block
   PrepLayout lay[CAP];
   PrepSum sum[CAP];
@@ -762,6 +981,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
   const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   for (int li = 0; li < p.n_layout; ++li) {
     const PrepLayout& L = p.lay[li];
+    if (L.i8) continue;  // phase (2b)
     const int groups_per_chunk = L.kc / 8;
     const int64_t total = int64_t(L.n_kc) * groups_per_chunk * M;
     for (int64_t i = tid; i < total; i += stride) {
@@ -784,6 +1004,158 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
                           ((int64_t(s * L.w8 + q) * M + m) * 4 + t) * 16;
       if (MQ_IN_BOUNDS(off + 16 <= int64_t(L.n_kc) * M * L.kc * 2, p.err))
         *reinterpret_cast<uint4*>(L.xf + off) = v;
+    }
+  }
+  // (2b) digit blocks of the integer kinds (one batch row): one warp per
+  // (unit, digit g). Every warp of a unit reads all its inputs to find the
+  // largest top exponent E and whether the digits hold every input exactly;
+  // lane l then writes digit g of the 16 inputs of slot group l = (s, jj, t).
+  // An input x = +-m 2^f (m < 256 an integer, f = e - 134 for a normal bf16 of
+  // biased exponent e, -133 for a subnormal) becomes X = m 2^(f + 48 - E),
+  // below 2^49, an integer when f >= E - 48; digit g is (X >> 7g) & 127 with
+  // x's sign. A unit with f < E - 48 somewhere, a non-finite input or E
+  // outside [-78, 100] gets the width's bf16 fragments and offset sum instead
+  // (written by the digit-0 warp).
+  if (p.n_i8 > 0) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = stride / 32;
+    constexpr int kNone = -100000;
+    for (int64_t wi = tid / 32; wi < int64_t(p.n_i8) * kI8Digits; wi += warps) {
+      const int g = static_cast<int>(wi % kI8Digits);
+      int64_t rem = wi / kI8Digits;
+      int li = 0;
+      while (!p.lay[li].i8 || rem >= p.lay[li].n_kc) {
+        if (p.lay[li].i8) rem -= p.lay[li].n_kc;
+        ++li;
+      }
+      const PrepLayout& L = p.lay[li];
+      const int r = L.i8, KC = L.kc, cpc = 128 / r;  // codes per unit, per 16-byte chunk
+      const int kc = static_cast<int>(rem);
+      const int64_t kbase = int64_t(kc) * KC;
+      const uint16_t* xr = reinterpret_cast<const uint16_t*>(L.x);  // one batch row
+      // (a) E, the smallest exponent f and non-finite inputs over the unit
+      int emax = kNone, fmin = 1 << 30;
+      bool bad = false;
+      const int ept = KC / 32;  // 4, 8 or 16 consecutive inputs per lane (K % 128 == 0: all in or all out)
+      const int64_t k0 = kbase + int64_t(lane) * ept;
+      uint32_t xe[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (k0 < L.K) {  // all loads first
+        if (ept == 16) {
+          const uint4 va = *reinterpret_cast<const uint4*>(xr + k0);
+          const uint4 vb = *reinterpret_cast<const uint4*>(xr + k0 + 8);
+          xe[0] = va.x; xe[1] = va.y; xe[2] = va.z; xe[3] = va.w;
+          xe[4] = vb.x; xe[5] = vb.y; xe[6] = vb.z; xe[7] = vb.w;
+        } else if (ept == 8) {
+          const uint4 va = *reinterpret_cast<const uint4*>(xr + k0);
+          xe[0] = va.x; xe[1] = va.y; xe[2] = va.z; xe[3] = va.w;
+        } else {
+          const uint2 va = *reinterpret_cast<const uint2*>(xr + k0);
+          xe[0] = va.x; xe[1] = va.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {  // zero words (past ept or past K) add nothing
+        const uint32_t bits = (u & 1) ? (xe[u >> 1] >> 16) : (xe[u >> 1] & 0xFFFFu);
+        const uint32_t ef = (bits >> 7) & 0xFFu, mf = bits & 0x7Fu;
+        if (ef == 0xFFu) bad = true;
+        if (ef == 0u && mf == 0u) continue;
+        const uint32_t m = ef ? (0x80u | mf) : mf;
+        const int f = static_cast<int>(ef ? ef : 1u) - 134;
+        emax = max(emax, f + 31 - __clz(static_cast<int>(m)));
+        fmin = min(fmin, f);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+        fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
+      }
+      const int E = emax == kNone ? 0 : emax;
+      if (emax != kNone && (fmin < E - 48 || E > 100 || E < -78)) bad = true;
+      const bool fallback = __any_sync(0xffffffffu, bad);
+      uint8_t* blk = L.xf + int64_t(kc) * i8_unit_bytes(r);
+      const int64_t blk_end = int64_t(L.n_kc) * i8_unit_bytes(r);  // bytes of the layout
+      if (!fallback) {
+        // (b) digit g of slot group (s, jj, t): MMAs j = 2 jj, 2 jj + 1 of chunk
+        // 4s + t, whose 16 inputs are the chunk's codes 16 jj .. 16 jj + 15
+        // (loaded at once), in the k-slot order of i8_regs
+        const int J2 = 16 / r / 2;
+        if (lane < 8 * J2) {
+          const int s = lane / (4 * J2), jj = (lane / 4) % J2, t = lane % 4;
+          const int64_t k16 = kbase + int64_t(4 * s + t) * cpc + 16 * jj;
+          uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          if (k16 < L.K) {  // the chunk lies wholly inside or outside K (K % 128 == 0)
+            const uint4 va = *reinterpret_cast<const uint4*>(xr + k16);
+            const uint4 vb = *reinterpret_cast<const uint4*>(xr + k16 + 8);
+            xw[0] = va.x; xw[1] = va.y; xw[2] = va.z; xw[3] = va.w;
+            xw[4] = vb.x; xw[5] = vb.y; xw[6] = vb.z; xw[7] = vb.w;
+          }
+          uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int b = 0; b < 16; ++b) {
+            const int h = b / 8, bb = b % 8;  // MMA 2 jj + h, k-slot byte bb
+            // the input's index among the 16: r = 8 bytes in order; r = 4
+            // codes 0, 4, 1, 5, 2, 6, 3, 7 of word 2 jj + h; r = 2 codes
+            // 4h + (0, 8, 1, 9, 2, 10, 3, 11) of word jj
+            const int u = r == 8 ? 8 * h + bb
+                        : r == 4 ? 8 * h + ((bb & 1) ? 4 : 0) + (bb >> 1)
+                                 : 4 * h + ((bb & 1) ? 8 : 0) + (bb >> 1);
+            const uint32_t bits = (u & 1) ? (xw[u >> 1] >> 16) : (xw[u >> 1] & 0xFFFFu);
+            const uint32_t ef = (bits >> 7) & 0xFFu, mf = bits & 0x7Fu;
+            const uint32_t m = ef ? (0x80u | mf) : mf;
+            const int sh = static_cast<int>(ef ? ef : 1u) - 134 + 48 - E - 7 * g;  // X >> 7g = m 2^sh
+            // m < 2^8: digit g = (m 2^sh) & 127 for sh in (-8, 7), else 0
+            uint32_t d = 0u;
+            if (sh >= 0) d = sh < 7 ? ((m << sh) & 127u) : 0u;
+            else d = sh > -8 ? ((m >> -sh) & 127u) : 0u;
+            const uint32_t sd = (bits & 0x8000u) ? (0u - d) & 0xFFu : d;
+            out[b >> 2] |= sd << (8 * (b & 3));
+          }
+          const int64_t off = kI8Header + (int64_t((s * J2 + jj) * 4 + t) * kI8Digits + g) * 16;
+          if (MQ_IN_BOUNDS(int64_t(kc) * i8_unit_bytes(r) + off + 16 <= blk_end, p.err))
+            *reinterpret_cast<uint4*>(blk + off) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        if (g == 0 && lane == 0) {
+          reinterpret_cast<int*>(blk)[0] = 0;
+          reinterpret_cast<int*>(blk)[1] = E;
+          reinterpret_cast<float*>(blk)[2] = 0.f;
+        }
+      } else if (g == 0) {
+        // (c) the width's bf16 fragments: group q of 8 inputs of chunk 4s + t at
+        // ((s W8 + q) 4 + t) 16, byte planes (r = 8) pairing codes (c0, c2), (c1, c3)
+        const int W8 = 16 / r;
+        float part = 0.f;
+        for (int grp = lane; grp < KC / 8; grp += 32) {
+          const int s = grp / (4 * W8), t = (grp / W8) % 4, q = grp % W8;
+          const int64_t kg = kbase + int64_t(4 * s + t) * cpc + 8 * q;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (kg < L.K) v = *reinterpret_cast<const uint4*>(xr + kg);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float xv = __uint_as_float(((u & 1) ? (w4[u >> 1] >> 16) : (w4[u >> 1] & 0xFFFFu)) << 16);
+            // the bf16 path's magic offset of input kg + u: 16 at r = 4, the
+            // class magics (k >> 1) & 7 at r = 2, none at r = 8 (kg % 8 == 0)
+            constexpr float kMagic2[kClasses] = {64.f, 16.f, 4.f, 64.f, 16.f, 4.f, 64.f, 16.f};
+            const float off = r == 4 ? 16.f : r == 2 ? kMagic2[((kg + u) >> 1) & 7] : 0.f;
+            part = fmaf(xv, off, part);
+          }
+          if (r == 8) {
+            const uint32_t a = __byte_perm(v.x, v.y, 0x5410), b = __byte_perm(v.x, v.y, 0x7632);
+            const uint32_t c = __byte_perm(v.z, v.w, 0x5410), d = __byte_perm(v.z, v.w, 0x7632);
+            v = make_uint4(a, b, c, d);
+          }
+          const int64_t off = kI8Header + int64_t((s * W8 + q) * 4 + t) * 16;
+          if (MQ_IN_BOUNDS(int64_t(kc) * i8_unit_bytes(r) + off + 16 <= blk_end, p.err))
+            *reinterpret_cast<uint4*>(blk + off) = v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) {
+          reinterpret_cast<int*>(blk)[0] = 1;
+          reinterpret_cast<int*>(blk)[1] = E;
+          reinterpret_cast<float*>(blk)[2] = part;
+        }
+      }
     }
   }
   // (4) Extra Precision sums: one warp per (job, row). With M' the next power
@@ -943,13 +1315,19 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
 // decode and MMA work grows with the codes in it: per-unit times of
 // single-width stacks on B200 at M = 1 put r = 4 at about 1.26x and r = 2 at
 // about 1.88x an r = 8 unit; r = 3 and 6 are scaled from their planes.
-int64_t unit_cost(const LinearJob& j) {
-  switch (decode_kind(j)) {
+int64_t unit_cost(int dk) {
+  switch (dk) {
     case 8: return 100;
     case 4: return 126;
     case 2: return 188;
     case 6: return 183;
     case 10: case 11: return 110;  // one 8-bit plane, one MMA per 16 codes, more decode work
+    // the integer kinds, from per-unit times of single-width stacks at one
+    // batch row on B200 (r = 8 streams near the HBM peak; r = 4 1.15x,
+    // r = 2 1.51x its unit time)
+    case kDkI8 + 8: return 100;
+    case kDkI8 + 4: return 115;
+    case kDkI8 + 2: return 151;
     default: return 301;  // 3
   }
 }
@@ -968,7 +1346,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
 
   // Distinct inputs (class sums) and distinct (input, layout) pairs. Few
   // entries: linear scans are cheaper than maps here.
-  struct LayoutInfo { const void* x; int b0, K, kc, w8, n_kc; size_t off; };
+  struct LayoutInfo { const void* x; int b0, i8, K, kc, w8, n_kc; uint32_t xunit; size_t off; };
   LayoutInfo layouts[CAP];
   const void* sum_x[CAP];
   int sum_k[CAP];
@@ -977,6 +1355,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   bool two_planes = false;
   int units = 0;
   size_t xf_bytes = 0;
+  uint32_t x_unit_max = 0;
   for (int i = 0; i < n_jobs; ++i) {
     const LinearJob& j = jobs[i];
     int b0, b1;
@@ -984,16 +1363,21 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     if (b1) two_planes = true;
     const int kc = P0 * 8 / b0;
     const int n_kc = static_cast<int>((j.K + kc - 1) / kc);
+    // planes of width 8, 4, 2 at one batch row run on the integer tensor cores
+    const int dk0 = decode_kind(j);
+    const int i8 = (M == 1 && (dk0 == 8 || dk0 == 4 || dk0 == 2)) ? dk0 : 0;
     int si = 0;
     while (si < n_sums && sum_x[si] != j.x) ++si;
     if (si == n_sums) { sum_x[n_sums] = j.x; sum_k[n_sums] = static_cast<int>(j.K); ++n_sums; }
     sum_of[i] = si;
     int li = 0;
-    while (li < n_layouts && !(layouts[li].x == j.x && layouts[li].b0 == b0)) ++li;
+    while (li < n_layouts && !(layouts[li].x == j.x && layouts[li].b0 == b0 && layouts[li].i8 == i8)) ++li;
     if (li == n_layouts) {
-      layouts[n_layouts++] = {j.x, b0, static_cast<int>(j.K), kc, (128 / b0) / 8, n_kc, xf_bytes};
-      xf_bytes += size_t(n_kc) * M * kc * 2;
+      const uint32_t xunit = i8 ? i8_unit_bytes(i8) : static_cast<uint32_t>(M * kc * 2);
+      layouts[n_layouts++] = {j.x, b0, i8, static_cast<int>(j.K), kc, (128 / b0) / 8, n_kc, xunit, xf_bytes};
+      xf_bytes += size_t(n_kc) * xunit;
       xf_bytes = (xf_bytes + 255) & ~size_t(255);
+      if (xunit > x_unit_max) x_unit_max = xunit;
     }
     lay_of[i] = li;
     const int nrb = static_cast<int>((j.N + RU - 1) / RU);
@@ -1006,7 +1390,8 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     d.N = static_cast<int>(j.N);
     d.K = static_cast<int>(j.K);
     d.r = j.r;
-    d.dk = decode_kind(j);
+    d.dk = i8 ? kDkI8 + i8 : dk0;
+    d.xunit = layouts[li].xunit;
     d.epc = nullptr;  // set with the workspace below
     d.kc = kc;
     d.n_kc = n_kc;
@@ -1068,8 +1453,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   const int P1 = two_planes ? P0 / 2 : 0;
   const uint32_t off_plane1 = static_cast<uint32_t>(RU * P0);
   const uint32_t off_x = off_plane1 + static_cast<uint32_t>(RU * P1);
-  const uint32_t x_bytes = static_cast<uint32_t>(M * (P0 * 8 / 2) * 2);  // largest KC (b0 = 2)
-  uint32_t stage_bytes = off_x + x_bytes;
+  uint32_t stage_bytes = off_x + x_unit_max;
   stage_bytes = (stage_bytes + 1023) & ~1023u;  // swizzled boxes start 1024-aligned
   int stages = static_cast<int>(kStageBudget / stage_bytes);
   stages = std::max(2, std::min(stages, kMaxStages));
@@ -1088,7 +1472,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   int64_t total_cost = 0;
   for (int i = 0; i < n_jobs; ++i) {
     const int64_t lin_units = (i + 1 < n_jobs ? gp.lin[i + 1].unit_begin : units) - gp.lin[i].unit_begin;
-    total_cost += lin_units * unit_cost(jobs[i]);
+    total_cost += lin_units * unit_cost(gp.lin[i].dk);
   }
   int n_zero = 0;
   {
@@ -1099,7 +1483,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
       // first unit whose preceding cost reaches the target
       while (li < n_jobs) {
         const int64_t lin_units = (li + 1 < n_jobs ? gp.lin[li + 1].unit_begin : units) - gp.lin[li].unit_begin;
-        const int64_t lin_cost = lin_units * unit_cost(jobs[li]);
+        const int64_t lin_cost = lin_units * unit_cost(gp.lin[li].dk);
         if (target <= cost_before + lin_cost) break;
         cost_before += lin_cost;
         ++li;
@@ -1108,7 +1492,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
       if (li >= n_jobs) {
         u = units;
       } else {
-        const int64_t w = unit_cost(jobs[li]);
+        const int64_t w = unit_cost(gp.lin[li].dk);
         u = gp.lin[li].unit_begin + static_cast<int>((target - cost_before + w - 1) / w);
       }
       if (c == 0) u = 0;
@@ -1140,10 +1524,12 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   pp.n_sum = n_sums;
   pp.n_zero = n_zero;
   pp.rows = RU;
+  pp.n_i8 = 0;
   for (int i = 0; i < n_layouts; ++i) {
     pp.lay[i] = {static_cast<const __nv_bfloat16*>(layouts[i].x), wsb + layouts[i].off,
                  layouts[i].K, layouts[i].kc, layouts[i].w8, layouts[i].n_kc,
-                 layouts[i].b0 == 8 ? 1 : 0};
+                 layouts[i].b0 == 8 ? 1 : 0, layouts[i].i8};
+    if (layouts[i].i8) pp.n_i8 += layouts[i].n_kc;
   }
   for (int i = 0; i < n_sums; ++i) {
     pp.sum[i] = {static_cast<const __nv_bfloat16*>(sum_x[i]),
@@ -1151,6 +1537,8 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   }
   int prep_grid = std::max(n_sums * M, sms);
   if (pp.n_ep > 0) prep_grid = 4 * sms;  // the Extra Precision gathers want many warps in flight
+  // one warp per (unit, digit) of the digit layouts, all in one round
+  prep_grid = std::max(prep_grid, (pp.n_i8 * kI8Digits + 7) / 8);
   prep_grid = std::min(prep_grid, 4 * sms);
   e = launch_pdl(gemv_prep_kernel<CAP>, dim3(prep_grid), dim3(256), 0, stream, pp);
   if (e != cudaSuccess) return e;
@@ -1185,15 +1573,19 @@ cudaError_t run_gemv(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stre
 }
 
 size_t gemv_scratch_bytes(const LinearJob& job, int M) {
-  // Same arithmetic as the planner in run_gemv_cap for one linear.
+  // Same arithmetic as the planner in run_gemv_cap for one linear (without an
+  // Extra Precision list): activation blocks, class sums, the trailing 256.
   const int P0 = tiling_p0(M);
   int b0, b1;
   job_planes(job, b0, b1);
   const int kc = P0 * 8 / b0;
   const int64_t n_kc = (job.K + kc - 1) / kc;
-  size_t xf = size_t(n_kc) * M * kc * 2;
+  const int dk = decode_kind(job);
+  const bool i8 = M == 1 && (dk == 8 || dk == 4 || dk == 2);
+  size_t xf = size_t(n_kc) * (i8 ? size_t(i8_unit_bytes(dk)) : size_t(M) * kc * 2);
   xf = (xf + 255) & ~size_t(255);
-  return xf + size_t(M) * kClasses * sizeof(float) + 256;
+  const size_t sums = (size_t(M) * kClasses * sizeof(float) + 255) & ~size_t(255);
+  return xf + sums + 256;
 }
 
 cudaError_t run_gemv_fixed_n(const LinearJob* jobs, int n_jobs, int M, cudaStream_t stream,

@@ -1,6 +1,6 @@
 // Device-side helpers for sm_100a: mbarriers, 1-D bulk (TMA) copies,
-// programmatic dependent launch, the legacy bf16 tensor-core MMA and a
-// nanosecond timer for bounded waits.
+// programmatic dependent launch, the legacy bf16 and u8 x s8 tensor-core
+// MMAs and a nanosecond timer for bounded waits.
 #pragma once
 
 #include <cstdint>
@@ -148,6 +148,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A(16x32 u8, row) * B(32x8 s8, col) + C, int32 accumulate (exact while
+// the sums fit). Fragments of the 8-bit m16n8k32 shape: a0 holds row g,
+// k = 4t..4t+3 (one byte each); a1 row g+8, same k; a2, a3 the same rows at
+// k + 16 (g = lane / 4, t = lane % 4); b0 = B[4t..4t+3][g], b1 = B[16+4t..][g].
+// D element (row, col) sits in thread (row % 8, col / 2), register
+// 2 (row / 8) + col % 2. On B200 this runs natively on the tensor cores' integer
+// path, one instruction per MMA.
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 

@@ -122,6 +122,12 @@ struct FixedScratch {
   size_t bytes;
   uint32_t* err;
 };
+// Reads and clears the wait-error word of mq_linear_noalloc's fixed array on
+// the current device (0 if that entry point never ran there).
+cudaError_t noalloc_take_error(uint32_t* flags);
+// The per-device error word if it exists already (null otherwise); never
+// allocates.
+uint32_t* find_error_word();
 // Scratch bytes the decode path needs for one linear at batch M.
 size_t gemv_scratch_bytes(const LinearJob& job, int M);
 // Decode path for one linear on caller-provided scratch; returns
@@ -143,6 +149,9 @@ cudaError_t run_gemv_fixed_n(const LinearJob* jobs, int n_jobs, int M, cudaStrea
 // Chained decoder stack (mq_chain_forward): scratch bytes, and the run, with
 // graph capture and replay of repeated identical calls when `use_graph`.
 size_t chain_scratch_bytes(int64_t M, int64_t D, int64_t Dkv, int64_t F);
+// Offsets of the last layer's intermediates (xn, qkv, a, o, h1, xn1, g, u,
+// act, down) inside the chain's scratch.
+void chain_views(int64_t M, int64_t D, int64_t Dkv, int64_t F, size_t out[10]);
 cudaError_t run_chain(const struct mq_chain_layer* layers, int n_layers, int M, int D, int Dkv, int F,
                       int hd, float* h, void* scratch, bool use_graph, cudaStream_t stream);
 void release_chain_graphs();

@@ -62,6 +62,26 @@ mq_status noalloc_fail(mq_status s, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
+
+// Reads and clears the array's wait-error word on the current device (0 if
+// mq_linear_noalloc was never set up there: then nothing can have set it).
+// Synchronous; allocates nothing.
+cudaError_t noalloc_take_error(uint32_t* flags) {
+  *flags = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+    if (static_cast<size_t>(dev) < g_noalloc_addr.size()) p = g_noalloc_addr[dev];
+  }
+  if (!p) return cudaSuccess;
+  e = cudaMemcpy(flags, p, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess || *flags == 0) return e;
+  return cudaMemset(p, 0, sizeof(uint32_t));
+}
+
 }  // namespace mq
 
 using namespace mq;
@@ -90,7 +110,7 @@ extern "C" mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, cons
   if (need > have)
     return noalloc_fail(MQ_ERR_INVALID_ARG,
                         "mq_linear_noalloc: M=%lld, K=%lld needs %zu scratch bytes, more than the fixed "
-                        "%zu (M*K up to about 512 Ki elements fits)",
+                        "%zu (M*K up to 524288 fits; K up to 174592 at M = 1)",
                         (long long)M, (long long)K, need, have);
   void* base = nullptr;
   cudaError_t e = noalloc_base(&base);

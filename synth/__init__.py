@@ -8,7 +8,11 @@ receive the very same host arrays produced here and nothing else.
 Shapes and distributions follow the Matryoshka Quantization pages' model
 families (Gemma-2 2B / 9B and Mistral 7B shaped linears, FFN weights drawn
 N(0, 0.02^2) or heavy-tailed Student-t(4)*0.02, activations N(0, 1)).
-Every generator is numpy.random.Generator(PCG64(seed)).
+Every host generator is numpy.random.Generator(PCG64(seed)). The benchmark's
+multi-gigabyte stack is drawn on the device instead (device_gaussian_weights,
+device_activations: torch's seeded generator, the same laws), so that building
+it does not take minutes of host time; a test that checks that workload draws
+the same tensors again and copies the rows it samples to the host.
 """
 from __future__ import annotations
 
@@ -23,6 +27,8 @@ __all__ = [
     "WORKLOADS",
     "mixnmatch_widths",
     "stack_shapes",
+    "device_gaussian_weights",
+    "device_activations",
 ]
 
 
@@ -146,3 +152,20 @@ def stack_shapes(n_layers: int = 32):
         for j, (name, n, k) in enumerate(mats):
             res.append((l, name, n, k, 1000 + 5 * l + j))
     return res
+
+
+def device_gaussian_weights(n: int, k: int, seed: int, device, std: float = 0.02):
+    """N(0, std^2) n x k weights drawn on `device` by torch's generator seeded
+    with `seed`, rounded to a bf16 tensor (the benchmark stack's weights)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    return (torch.randn((n, k), generator=gen, device=device) * std).to(torch.bfloat16)
+
+
+def device_activations(m: int, k: int, seed: int, device):
+    """N(0, 1) activations, m x k, drawn on `device` (seeded), as a bf16 tensor."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    return torch.randn((m, k), generator=gen, device=device).to(torch.bfloat16)

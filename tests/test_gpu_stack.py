@@ -67,3 +67,39 @@ def test_7b_shaped_stack_sampled_rows():
         x_vals = synth.f32_from_bf16_bits(xs_bits[k]).astype(np.float64)
         check_linear(y[:, rows], x_vals, oracle.dequant_slice(q, a, z, widths[layer]),
                      f"layer {layer} {n}x{k}")
+
+
+def test_bench_workload_every_linear_sampled_rows():
+    """The benchmark's own configuration, in its own launch: the 32-layer
+    7B-shaped Mix'n'Match stack (160 linears, widths 8 / 4 / 2 by layer) at
+    one batch row, built and stepped by bench.Stack exactly as the timed loop
+    does. Every output must be written; on 24 sampled weight rows of every
+    linear (first, last and random rows, so both whole and CTA-shared row
+    blocks are hit) y must match the oracle, which quantizes the same rows of
+    the same seeded weights on the host."""
+    import bench
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stack = bench.Stack(1, dev)
+    assert len(stack.lins) == 160 and stack.widths == synth.mixnmatch_widths(32)
+    stack.y_all.fill_(float("nan"))
+    s = torch.cuda.current_stream(dev)
+    stack.step(s)
+    torch.cuda.synchronize()
+    mq.device_status()
+    assert bool(torch.isfinite(stack.y_all).all()), "an output element was not written"
+    xs = {k: synth.f32_from_bf16_bits(v.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+          for k, v in stack.x.items()}
+    rng = np.random.default_rng(5)
+    mats = synth.WORKLOADS["mixnmatch_7b_stack"]["mats"]
+    worst = 0.0
+    for i, (x, p, a, z, y, n, k) in enumerate(stack.lins):
+        layer, j = divmod(i, len(mats))
+        w = synth.device_gaussian_weights(n, k, stack.seed_base + 5 * layer + j, dev)
+        rows = np.unique(np.concatenate([[0, n - 1], rng.choice(n, size=22, replace=False)]))
+        w_rows = w[torch.from_numpy(rows).to(dev)].view(torch.int16).cpu().numpy().view(np.uint16)
+        q, a_r, z_r = oracle.quantize_minmax(synth.f32_from_bf16_bits(w_rows).astype(np.float64))
+        y_rows = y[:, torch.from_numpy(rows).to(dev)].cpu().numpy().astype(np.float64)
+        worst = max(worst, check_linear(y_rows, xs[k], oracle.dequant_slice(q, a_r, z_r, stack.widths[layer]),
+                                        f"bench stack linear {i} (layer {layer}) {n}x{k}"))
+    print(f"bench workload: worst err/tol {worst:.3f}")
