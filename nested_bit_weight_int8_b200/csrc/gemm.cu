@@ -4,11 +4,13 @@
 // Interpolative Slicing" for the widths 6 and 3 served from the same int8
 // container).
 //
-// With codes c[n,k] = S(q[n,k], r) / 2^(8-r), the product factors as
-//   y[m,n] = A_n * sum_k x[m,k] c[n,k] - B_n * Sx[m],
-//   A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n,  Sx[m] = sum_k x[m,k],
-// so the contraction runs on exact integer operands: every code is an
-// integer below 256, exact in bf16, and products and sums are fp32.
+// With codes c[n,k] = S(q[n,k], r) / 2^(8-r) and c0_n the code nearest to
+// z_n / 2^(8-r), the product factors as
+//   y[m,n] = A_n * sum_k x[m,k] (c[n,k] - c0_n) - B_n * Sx[m],
+//   A_n = alpha_n 2^(8-r),  B_n = alpha_n (z_n - c0_n 2^(8-r)),  Sx[m] = sum_k x[m,k],
+// so the contraction runs on exact integer operands (c - c0 lies in
+// [-255, 255], exact in bf16; products and sums are fp32), and the sums stay
+// small where the dequantized weights are small.
 //
 // Tile: 128 weight rows (n) x 256 batch rows (m), K in stages of 64 codes.
 // The weights are the MMA's A operand and live in tensor memory; x is the B
@@ -96,21 +98,25 @@ __global__ void __launch_bounds__(256) rowsum_kernel(const __nv_bfloat16* __rest
 
 // ------------------------------------------------------------ decode
 // bf16x2 128.0 in both halves: OR-ing a code c < 128 into the mantissa gives
-// 128 + c exactly; subtracting 128 again leaves the integer c.
+// 128 + c exactly. Each decode thread owns one weight row and subtracts
+// 128 + c0 of that row, c0 the code nearest to the row's zero point (sub2),
+// which leaves the integer c - c0: the MMA then sums x (c - c0), small where
+// the dequantized weights are small, instead of x c.
 constexpr uint32_t kMag128x2 = 0x43004300u;
 
-__device__ __forceinline__ uint32_t exact_pair(uint32_t codes2) {
+__device__ __forceinline__ uint32_t exact_pair(uint32_t codes2, uint32_t sub2) {
   uint32_t d;
   // bf16x2 subtract (exact: both operands and the result are small integers)
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(codes2 | kMag128x2), "r"(kMag128x2));
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(codes2 | kMag128x2), "r"(sub2));
   return d;
 }
 
-// Two container bytes (0..255) as an exact bf16x2 pair, through fp32:
-// 2^23 + c is built by placing c in the low mantissa byte.
-__device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
-  const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - 8388608.0f;
-  const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - 8388608.0f;
+// Two container bytes (0..255) minus c0 as an exact bf16x2 pair, through
+// fp32: 2^23 + c is built by placing c in the low mantissa byte, and subf =
+// 2^23 + c0 is subtracted.
+__device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo, uint32_t sel_hi, float subf) {
+  const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - subf;
+  const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - subf;
   const __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
   return *reinterpret_cast<const uint32_t*>(&b);
 }
@@ -126,8 +132,8 @@ __device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo
 // bits in both halves after the shift by s).
 template <int R>
 __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, const uint8_t* p1,
-                                         uint32_t (&v)[16], uint32_t h2 = 0, uint32_t kmask = 0,
-                                         int sh = 0) {
+                                         uint32_t (&v)[16], uint32_t sub2, float subf, uint32_t h2 = 0,
+                                         uint32_t kmask = 0, int sh = 0) {
   if constexpr (R == 10 || R == 11) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint4 b = *reinterpret_cast<const uint4*>(p0b);
@@ -137,18 +143,18 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
       // codes 2j, 2j+1 are bytes (0, 1) or (2, 3) of word j / 2
       const uint32_t t = __byte_perm(w[j / 2], 0u, (j % 2 == 0) ? 0x4140u : 0x4342u);
       const uint32_t u = (R == 10) ? __viaddmin_u16x2(t, h2, 0x00FF00FFu) : t + h2;
-      v[j] = exact_pair((u >> sh) & kmask);
+      v[j] = exact_pair((u >> sh) & kmask, sub2);
     }
   } else if constexpr (R == 2) {
     const uint2 a = *reinterpret_cast<const uint2*>(p0);
     const uint32_t w[2] = {a.x, a.y};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u);
+    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u, sub2);
   } else if constexpr (R == 4) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu);
+    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu, sub2);
   } else if constexpr (R == 3) {
     const uint2 a = *reinterpret_cast<const uint2*>(p0);
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p1);
@@ -157,7 +163,7 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     for (int j = 0; j < 16; ++j) {
       const uint32_t lo = (w[j / 8] >> (2 * (j % 8))) & 0x00030003u;
       const uint32_t hi = ((u >> j) & 0x00010001u) << 2;
-      v[j] = exact_pair(lo | hi);
+      v[j] = exact_pair(lo | hi, sub2);
     }
   } else if constexpr (R == 6) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
@@ -168,7 +174,7 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     for (int j = 0; j < 16; ++j) {
       const uint32_t lo = (w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu;
       const uint32_t hi = ((u[j / 8] >> (2 * (j % 8))) & 0x00030003u) << 4;
-      v[j] = exact_pair(lo | hi);
+      v[j] = exact_pair(lo | hi, sub2);
     }
   } else {  // R == 8: bytes, 4 codes per word
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
@@ -176,8 +182,8 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      v[j] = (j % 2 == 0) ? exact_pair_bytes(w[j / 2], 0x7440u, 0x7441u)
-                          : exact_pair_bytes(w[j / 2], 0x7442u, 0x7443u);
+      v[j] = (j % 2 == 0) ? exact_pair_bytes(w[j / 2], 0x7440u, 0x7441u, subf)
+                          : exact_pair_bytes(w[j / 2], 0x7442u, 0x7443u, subf);
   }
 }
 
@@ -303,6 +309,17 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
     const uint32_t ch2 = (R >= 10) ? (1u << (cs - 1)) * 0x10001u : 0u;
     const uint32_t ckm = (R >= 10) ? ((1u << (R == 10 ? p.r : p.r + 1)) - 1u) * 0x10001u : 0u;
     constexpr int b1 = (R == 3) ? 1 : (R == 6) ? 2 : 0;
+    // c0, the code nearest to this row's zero point (clamped to the code
+    // range): the decode subtracts it and the epilogue adds alpha c0 2^s back
+    const int rw = R >= 10 ? p.r : R;
+    const int cmax = R == 11 ? (1 << rw) : (1 << rw) - 1;
+    int c0 = 0;
+    if (n0 + row < p.N) {
+      const float zc = rintf(__ldg(p.zero + n0 + row) * (1.0f / static_cast<float>(1 << (8 - rw))));
+      c0 = zc <= 0.f ? 0 : zc >= static_cast<float>(cmax) ? cmax : static_cast<int>(zc);
+    }
+    const uint32_t sub2 = (0x4300u | static_cast<uint32_t>(c0 & 0x7F)) * 0x10001u;  // 128 + c0 (c0 < 128)
+    const float subf = 8388608.0f + static_cast<float>(c0);
     bool ok = true;
     for (int it = grp; it < n_k; it += 2) {
       const int s = it % kStages;
@@ -344,7 +361,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       (void)st_end;  // read only by the debug build's checks
       // (r1 is read only by widths with a second plane)
       if (MQ_IN_BOUNDS(r0 + 16 <= st_end && r0b + 16 <= st_end && (b1 == 0 || r1 + 8 <= st_end), p.err))
-        decode32<R>(r0, r0b, r1, v, ch2, ckm, cs);
+        decode32<R>(r0, r0b, r1, v, sub2, subf, ch2, ckm, cs);
       tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();
@@ -361,9 +378,11 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       const bool row_ok = n < p.N;
       float A = 0.f, B = 0.f;
       if (row_ok) {
+        // y = A sum x (c - c0) - alpha (z - c0 2^s) Sx
         const float a = __ldg(p.alpha + n);
-        A = a * static_cast<float>(1 << (8 - (R >= 10 ? p.r : R)));
-        B = a * __ldg(p.zero + n);
+        const float sc = static_cast<float>(1 << (8 - rw));
+        A = a * sc;
+        B = a * (__ldg(p.zero + n) - static_cast<float>(c0) * sc);
       }
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {

@@ -40,13 +40,15 @@
 // the mantissa of a bf16 power of two 2^e at a bit position p, which yields
 // exactly 2^e + c * 2^(e-7+p); choosing p and e so that the code weight is 1
 // (or 4, 16 for the high plane of r = 3, 6) gives the integer value
-// off + weight*c, exact in bf16. A byte (r = 8) has one significant bit too
-// many for this; it goes through fp32 instead (below). The offsets "off"
-// sum to O_m = sum_k x[m,k] off(k), which depends only on k mod 16 and is
-// removed in the epilogue from per-class activation sums computed once:
-//   y = A_n (acc - O_m) - B_n Sx_m,  A_n = alpha_n 2^(8-r),  B_n = alpha_n z_n.
-// Offsets stay <= 272 (none at r = 8), so fp32 partial sums stay small
-// (accuracy), and two codes are decoded per LOP3 (issue budget at r = 2).
+// 2^e + weight*c, exact in bf16. One bf16x2 subtract then takes out the magic
+// 2^e and, on the low plane, the centre code 2^(r-1): the MMA sums
+// x (c - 2^(r-1)) with no offset, so an fp32 partial sum never carries a
+// magic (up to 256 per code) that the epilogue would have to cancel again, and
+// a row whose zero point sits near the middle of the codes keeps small sums.
+// A byte (r = 8) has one significant bit too many for the magic; it goes
+// through fp32 instead (below), with the same centring. The epilogue is
+//   y = A_n acc - alpha_n (z_n - 128) Sx_m,  A_n = alpha_n 2^(8-r),
+// since 2^(r-1) 2^(8-r) = 128 at every width.
 //
 // Slicing on load. A linear may also stream the int8 container itself (the
 // r = 8 plane) and slice each byte while decoding, so one stored matrix serves
@@ -85,7 +87,7 @@ constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
 // Decode kinds of the planes at one batch row on the integer tensor cores:
 // kDkI8 + r for r = 8, 4, 2. A unit is 256 rows x 128 plane bytes (1024 / r
 // codes). Its staged activation block is a 64-byte header (int mode: 0 digits,
-// 1 bf16 fragments; int E, the unit's largest exponent; float O, the offset
+// 1 bf16 fragments; int E, the unit's largest exponent; float Sxu, the input
 // sum of a bf16 unit) and then slot (s, jj, t, g) of 16 bytes at
 // 64 + (((s * J / 2 + jj) * 4 + t) * kI8Digits + g) * 16, J = 16 / r MMAs per
 // 16-byte chunk: digit g of the 16 inputs of MMAs 2 jj and 2 jj + 1 of chunk
@@ -167,6 +169,14 @@ template <> struct Geo<6> { static constexpr int b0 = 4, b1 = 2, W8 = 4; };
 template <> struct Geo<10> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
 template <> struct Geo<11> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
 
+// bf16x2 of a small positive integer v (at most 8 significant bits, exact)
+// in both halves.
+__host__ __device__ constexpr uint32_t bf16x2_int(int v) {
+  int e = 0;
+  while ((2 << e) <= v) ++e;
+  return ((static_cast<uint32_t>(127 + e) << 7) | ((static_cast<uint32_t>(v) << (7 - e)) & 0x7Fu)) * 0x10001u;
+}
+
 // Per-linear constants of the slice-on-load decode (both 16-bit halves):
 // h2 the rounding addend 2^(s-1), kmask the code's bits after the shift, mag
 // the bf16 power of two the code is OR-ed under (code weight 1).
@@ -202,6 +212,55 @@ __device__ __forceinline__ uint32_t shift_to(uint32_t w) {
   else return w >> SIG;
 }
 
+// a - b on bf16x2 pairs. The decode uses it on exact small integers (a code
+// under its magic, minus the magic and the centre code), where it is exact.
+__device__ __forceinline__ uint32_t bsub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// The centre code of a row: the code nearest to z / 2^(8-r), clamped to
+// [0, cmax]. The bf16 decode subtracts it from every code of the row and the
+// epilogue adds alpha c0 2^(8-r) back through the zero-point term, so the
+// MMA sums x (c - c0), small wherever the dequantized weights are small.
+__device__ __forceinline__ int centre_code(float z, int rw, int cmax) {
+  const float zc = rintf(z * (1.0f / static_cast<float>(1 << (8 - rw))));
+  return zc <= 0.f ? 0 : zc >= static_cast<float>(cmax) ? cmax : static_cast<int>(zc);
+}
+
+// What the bf16 decode subtracts from one weight row's registers: s[i] =
+// bf16x2 of magic_i + c0 for the low plane's magics (at most three classes),
+// f = 2^23 + c0 for bytes through fp32; c0 itself for the epilogue.
+struct RowSub {
+  uint32_t s[3];
+  float f;
+  float c0;
+};
+
+template <int R>
+__device__ __forceinline__ RowSub make_rowsub(const float* zero, int n, int N, int r) {
+  const int rw = (R == 10 || R == 11) ? r : R;
+  const int cmax = R == 11 ? (1 << rw) : (1 << rw) - 1;
+  const int c0 = n < N ? centre_code(zero[n], rw, cmax) : 0;
+  // the low plane's magics: r = 2 by bit position 1, 3, 5; r = 3 by 3, 5;
+  // r = 4 and 6 one; the container the power of two 2^r (Eq. 6) or 2^(r+1)
+  const int m0 = R == 2 ? 64 : (R == 3 || R == 4 || R == 6) ? 16 : (R == 10 ? (1 << rw) : (2 << rw));
+  const int m1 = R == 2 ? 16 : 4;
+  const int m2 = 4;
+  auto pair = [](int v) {
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(static_cast<float>(v)));  // exact: v < 256
+    return b * 0x10001u;
+  };
+  RowSub rs;
+  rs.s[0] = pair(m0 + c0);
+  rs.s[1] = pair(m1 + c0);
+  rs.s[2] = pair(m2 + c0);
+  rs.f = 8388608.0f + static_cast<float>(c0);
+  rs.c0 = static_cast<float>(c0);
+  return rs;
+}
+
 // (a & mask) | magic in one LOP3: both constants travel in registers, so the
 // instruction needs no second immediate.
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic) {
@@ -218,37 +277,41 @@ constexpr uint32_t kMag4 = 0x40804080u, kMag8 = 0x41004100u, kMag16 = 0x41804180
 constexpr uint32_t kMaskP3b2 = 0x00180018u, kMaskP5b2 = 0x00600060u, kMaskP3b4 = 0x00780078u;
 
 // Two bytes of w (chosen by the byte_perm selectors, which put the byte under
-// the exponent of 2^23) as an exact bf16x2 pair of integers 0..255.
-__device__ __forceinline__ uint32_t bytes_bf16x2(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
-  const float lo = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - 8388608.0f;
-  const float hi = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - 8388608.0f;
+// the exponent of 2^23) minus the row's centre code c0 (subf = 2^23 + c0), as
+// an exact bf16x2 pair of integers -255..255.
+__device__ __forceinline__ uint32_t bytes_bf16x2(uint32_t w, uint32_t sel_lo, uint32_t sel_hi, float subf) {
+  const float lo = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_lo)) - subf;
+  const float hi = __uint_as_float(__byte_perm(w, 0x4B000000u, sel_hi)) - subf;
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
 
 // The pair of 2-bit codes at half-word position P (0, 2, ..., 14) of a plane
-// word as bf16x2. A left shift by 1 puts positions 0-4 at bits 1, 3, 5 of
-// each half, right shifts by 5 and 11 do the same for 6-10 and 12-14, so a
+// word as bf16x2 c - c0. A left shift by 1 puts positions 0-4 at bits 1, 3, 5
+// of each half, right shifts by 5 and 11 do the same for 6-10 and 12-14, so a
 // word costs three shifts and eight LOP3s. The code sits under the magic
-// 2^(7-p) that gives it weight 1: offsets 64, 16, 4 (the bits shifted in
-// from the other half fall outside the mask). An earlier form used shifts of
-// 0, 6, 12 and took the offset 128 of bit 0 out with a bf16x2 subtract: one
-// instruction more per word.
+// 2^(7-p) that gives it weight 1 (the bits shifted in from the other half
+// fall outside the mask); one bf16x2 subtract of the magic plus the row's
+// centre code c0 leaves c - c0.
 template <int P>
-__device__ __forceinline__ uint32_t pick2(uint32_t w) {
+__device__ __forceinline__ uint32_t pick2(uint32_t w, const RowSub& rs) {
   constexpr int sh = P <= 4 ? -1 : (P <= 10 ? 5 : 11);
   constexpr int p = P - sh;
   constexpr uint32_t mask = 0x00030003u << p;
-  return and_or(shift_to<sh>(w), mask, p == 1 ? kMag64 : p == 3 ? kMag16 : kMag4);
+  return bsub(and_or(shift_to<sh>(w), mask, p == 1 ? kMag64 : p == 3 ? kMag16 : kMag4),
+              rs.s[p == 1 ? 0 : p == 3 ? 1 : 2]);
 }
 
 // Decoded A registers of one MMA for one weight row: x0 fills k-slots
 // {2t, 2t+1}, x1 fills {2t+8, 2t+9}. PLANE 0 is the low plane, 1 the high
-// plane; Q is the 8-code group of the chunk, HF the 4-code half of it.
+// plane; Q is the 8-code group of the chunk, HF the 4-code half of it. Every
+// register holds exact integers with no offset: plane 0 its code minus the
+// row's centre code c0, plane 1 its weighted code, so the MMA sums x (c - c0)
+// and never carries the magics through fp32.
 template <int R, int PLANE, int Q, int HF>
 __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint32_t (&hi)[2],
-                                            const Cdec& cd, uint32_t& x0, uint32_t& x1) {
+                                            const Cdec& cd, const RowSub& rs, uint32_t& x0, uint32_t& x1) {
   if constexpr (R == 10 || R == 11) {
     // container bytes c0..c3 of one word, registers pair (c0, c2) and (c1, c3)
     // as the r = 8 plane does; q + h never leaves its 16-bit half
@@ -256,38 +319,38 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
     const uint32_t ev = w & 0x00FF00FFu;
     const uint32_t od = __byte_perm(w, 0u, 0x4341);
     if constexpr (R == 10) {
-      x0 = and_or(__viaddmin_u16x2(ev, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag);
-      x1 = and_or(__viaddmin_u16x2(od, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag);
+      x0 = bsub(and_or(__viaddmin_u16x2(ev, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag), rs.s[0]);
+      x1 = bsub(and_or(__viaddmin_u16x2(od, cd.h2, 0x00FF00FFu) >> 1, cd.kmask, cd.mag), rs.s[0]);
     } else {
-      x0 = and_or((ev + cd.h2) >> 2, cd.kmask, cd.mag);
-      x1 = and_or((od + cd.h2) >> 2, cd.kmask, cd.mag);
+      x0 = bsub(and_or((ev + cd.h2) >> 2, cd.kmask, cd.mag), rs.s[0]);
+      x1 = bsub(and_or((od + cd.h2) >> 2, cd.kmask, cd.mag), rs.s[0]);
     }
   } else if constexpr (R == 2) {
     // 2-bit codes, word = 16 codes; x0 holds codes 4j, 4j+1 (half-word
     // position 4j), x1 codes 4j+2, 4j+3 (position 4j+2), j = 2(Q%2)+HF.
     constexpr int j = 2 * (Q % 2) + HF;
-    x0 = pick2<4 * j>(lo[Q / 2]);
-    x1 = pick2<4 * j + 2>(lo[Q / 2]);
+    x0 = pick2<4 * j>(lo[Q / 2], rs);
+    x1 = pick2<4 * j + 2>(lo[Q / 2], rs);
   } else if constexpr (R == 3 && PLANE == 0) {
     // 2-bit codes, word = 16 codes; pairs 2j, 2j+1 (j = 2(Q%2)+HF) at half-bits
     // 4j, 4j+2 -> bits 3-4 (16 + c) and bits 5-6 (4 + c) after one shift.
     constexpr int j = 2 * (Q % 2) + HF;
     const uint32_t sh = shift_to<4 * j - 3>(lo[Q / 2]);
-    x0 = and_or(sh, kMaskP3b2, kMag16);
-    x1 = and_or(sh, kMaskP5b2, kMag4);
+    x0 = bsub(and_or(sh, kMaskP3b2, kMag16), rs.s[0]);
+    x1 = bsub(and_or(sh, kMaskP5b2, kMag4), rs.s[1]);
   } else if constexpr (R == 4 || (R == 6 && PLANE == 0)) {
     // 4-bit codes, word = 8 codes; pairs 2HF, 2HF+1 at half-bits 8HF, 8HF+4 -> bits 3-6 (16 + c)
     const uint32_t w = lo[Q];
-    x0 = and_or(shift_to<8 * HF - 3>(w), kMaskP3b4, kMag16);
-    x1 = and_or(shift_to<8 * HF + 1>(w), kMaskP3b4, kMag16);
+    x0 = bsub(and_or(shift_to<8 * HF - 3>(w), kMaskP3b4, kMag16), rs.s[0]);
+    x1 = bsub(and_or(shift_to<8 * HF + 1>(w), kMaskP3b4, kMag16), rs.s[0]);
   } else if constexpr (R == 8) {
     // bytes c0..c3 of one word; registers pair (c0, c2) and (c1, c3). A byte
     // has 8 significant bits, one more than a bf16 mantissa holds under a
-    // magic exponent, so it goes through fp32: 2^23 + c minus 2^23 is c, and
-    // its conversion to bf16 is exact. No offset remains.
+    // magic exponent, so it goes through fp32: 2^23 + c minus 2^23 + c0 is
+    // c - c0, and its conversion to bf16 is exact.
     const uint32_t w = lo[2 * Q + HF];
-    x0 = bytes_bf16x2(w, 0x7440u, 0x7442u);
-    x1 = bytes_bf16x2(w, 0x7441u, 0x7443u);
+    x0 = bytes_bf16x2(w, 0x7440u, 0x7442u, rs.f);
+    x1 = bytes_bf16x2(w, 0x7441u, 0x7443u, rs.f);
   } else if constexpr (R == 3) {
     // high 1-bit plane (weight 4), word = 32 codes; pairs P = 4(Q%4)+2HF, +1 at
     // half-bit P; one shift puts the group's 4 pairs at bits 3..6 (64/32/16/8 + 4h)
@@ -295,30 +358,13 @@ __device__ __forceinline__ void decode_quad(const uint32_t (&lo)[4], const uint3
     constexpr int p0 = 3 + 2 * HF;
     constexpr uint32_t m0 = (1u << p0) | (1u << (16 + p0));
     constexpr uint32_t m1 = (1u << (p0 + 1)) | (1u << (17 + p0));
-    x0 = and_or(sh, m0, HF == 0 ? kMag64 : kMag16);
-    x1 = and_or(sh, m1, HF == 0 ? kMag32 : kMag8);
+    x0 = bsub(and_or(sh, m0, HF == 0 ? kMag64 : kMag16), HF == 0 ? kMag64 : kMag16);
+    x1 = bsub(and_or(sh, m1, HF == 0 ? kMag32 : kMag8), HF == 0 ? kMag32 : kMag8);
   } else {  // R == 6, high 2-bit plane (weight 16), word = 16 codes
     constexpr int j = 2 * (Q % 2) + HF;
     const uint32_t sh = shift_to<4 * j - 3>(hi[Q / 2]);
-    x0 = and_or(sh, kMaskP3b2, kMag256);
-    x1 = and_or(sh, kMaskP5b2, kMag64);
-  }
-}
-
-// Offset of the decoded value per activation class (k >> 1) & 7 for each
-// width (the sum over the planes of the magic added to the code). The offsets
-// stay small next to the code unit (at most 32 at r = 2), so the fp32 sums
-// lose little to cancellation when the offsets are taken out again.
-__device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses]) {
-  constexpr float r2[kClasses] = {64.f, 16.f, 4.f, 64.f, 16.f, 4.f, 64.f, 16.f};
-  constexpr float r3[4] = {80.f, 36.f, 32.f, 12.f};
-  constexpr float r6[4] = {272.f, 80.f, 272.f, 80.f};
-  // the container sliced on load: one magic for every class
-  const float cont = static_cast<float>(1 << (dk == 10 ? r : r + 1));
-#pragma unroll
-  for (int i = 0; i < kClasses; ++i) {
-    // the integer kinds take each unit's offsets out when they fold it
-    c[i] = is_i8(dk) ? 0.f : dk >= 10 ? cont : r == 8 ? 0.f : r == 4 ? 16.f : r == 2 ? r2[i] : r == 3 ? r3[i & 3] : r6[i & 3];
+    x0 = bsub(and_or(sh, kMaskP3b2, kMag256), kMag256);
+    x1 = bsub(and_or(sh, kMaskP5b2, kMag64), kMag64);
   }
 }
 
@@ -327,8 +373,8 @@ __device__ __forceinline__ void offset_coeffs(int dk, int r, float (&c)[kClasses
 template <int R, int NT, int TW, int Q>
 __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, const Cdec& cd, uint32_t* errp,
-                                           float (&ch)[TW][NT][2][4]) {
+                                           int gbase, const Cdec& cd, const RowSub (&rs)[TW][2],
+                                           uint32_t* errp, float (&ch)[TW][NT][2][4]) {
   uint4 xb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -350,10 +396,10 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
 #pragma unroll
       for (int T = 0; T < TW; ++T) {
         uint32_t a0, a1, a2, a3;
-        if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 0, Q, 0>(lo[T][1], hi[T][1], cd, a1, a3); }
-        if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 1, Q, 0>(lo[T][1], hi[T][1], cd, a1, a3); }
-        if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 0, Q, 1>(lo[T][1], hi[T][1], cd, a1, a3); }
-        if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[T][0], hi[T][0], cd, a0, a2); decode_quad<R, 1, Q, 1>(lo[T][1], hi[T][1], cd, a1, a3); }
+        if (hf == 0 && pl == 0) { decode_quad<R, 0, Q, 0>(lo[T][0], hi[T][0], cd, rs[T][0], a0, a2); decode_quad<R, 0, Q, 0>(lo[T][1], hi[T][1], cd, rs[T][1], a1, a3); }
+        if (hf == 0 && pl == 1) { decode_quad<R, 1, Q, 0>(lo[T][0], hi[T][0], cd, rs[T][0], a0, a2); decode_quad<R, 1, Q, 0>(lo[T][1], hi[T][1], cd, rs[T][1], a1, a3); }
+        if (hf == 1 && pl == 0) { decode_quad<R, 0, Q, 1>(lo[T][0], hi[T][0], cd, rs[T][0], a0, a2); decode_quad<R, 0, Q, 1>(lo[T][1], hi[T][1], cd, rs[T][1], a1, a3); }
+        if (hf == 1 && pl == 1) { decode_quad<R, 1, Q, 1>(lo[T][0], hi[T][0], cd, rs[T][0], a0, a2); decode_quad<R, 1, Q, 1>(lo[T][1], hi[T][1], cd, rs[T][1], a1, a3); }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const uint32_t b0 = hf ? xb[nt].z : xb[nt].x;
@@ -368,15 +414,15 @@ __device__ __forceinline__ void group_mmas(const uint32_t (&lo)[TW][2][4], const
 template <int R, int NT, int TW, int... Qs>
 __device__ __forceinline__ void chunk_mmas(const uint32_t (&lo)[TW][2][4], const uint32_t (&hi)[TW][2][2],
                                            const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT],
-                                           int gbase, const Cdec& cd, uint32_t* errp,
-                                           float (&ch)[TW][NT][2][4],
+                                           int gbase, const Cdec& cd, const RowSub (&rs)[TW][2],
+                                           uint32_t* errp, float (&ch)[TW][NT][2][4],
                                            std::integer_sequence<int, Qs...>) {
-  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, cd, errp, ch), ...);
+  (group_mmas<R, NT, TW, Qs>(lo, hi, xaddr, xstep, gbase, cd, rs, errp, ch), ...);
 }
 
-// One staged unit for this warp's 16-row tiles. All sub-steps are unrolled
-// and their plane loads issued first. Sub-steps past the unit's valid codes
-// read zero-filled planes and zero activations and add nothing. Activation
+// One staged unit for this warp's 16-row tiles, sub-step by sub-step.
+// Sub-steps past the unit's valid codes read zero-filled planes and zero
+// activations and add nothing. Activation
 // group q of chunk 4s+t for batch row m sits at ((((s*W8 + q)*M + m)*4 + t)
 // * 16) bytes of the staged block; lanes whose batch row is past M read a
 // zero block instead (step 0). With 128-byte plane rows the box is stored in
@@ -385,16 +431,18 @@ template <int R, int NT>
 __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* st1,
                                              const uint32_t (&xaddr)[NT],
                                              const uint32_t (&xstep)[NT], int warp, int lane,
-                                             const Cdec& cd, uint32_t* errp,
-                                             float (&ch)[Tiling<NT>::TW][NT][2][4]) {
+                                             const Cdec& cd, const RowSub (&rs)[Tiling<NT>::TW][2],
+                                             uint32_t* errp, float (&ch)[Tiling<NT>::TW][NT][2][4]) {
   using G = Geo<R>;
   using TL = Tiling<NT>;
   constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0, P1 = TL::P0 / 2;
   const int g = lane >> 2, t = lane & 3;
-  uint32_t lo[NSUB][TW][2][4];
-  uint32_t hi[NSUB][TW][2][2];
+  // one sub-step's planes at a time (the row subtrahends take the registers
+  // a whole unit's words would)
 #pragma unroll
   for (int s = 0; s < NSUB; ++s) {
+    uint32_t lo[TW][2][4];
+    uint32_t hi[TW][2][2];
     const int ci = 4 * s + t;  // this thread's 16-byte chunk of the low plane
 #pragma unroll
     for (int T = 0; T < TW; ++T) {
@@ -403,20 +451,18 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
         const int row = warp * TL::RPW + 16 * T + g + 8 * h;
         const int cs = TL::SWZ ? (ci ^ (row & 7)) : ci;
         const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * P0 + cs * 16);
-        lo[s][T][h][0] = v.x; lo[s][T][h][1] = v.y; lo[s][T][h][2] = v.z; lo[s][T][h][3] = v.w;
+        lo[T][h][0] = v.x; lo[T][h][1] = v.y; lo[T][h][2] = v.z; lo[T][h][3] = v.w;
         if constexpr (G::b1 != 0) {
           const uint2 u = *reinterpret_cast<const uint2*>(st1 + row * P1 + ci * 8);
-          hi[s][T][h][0] = u.x; hi[s][T][h][1] = u.y;
+          hi[T][h][0] = u.x; hi[T][h][1] = u.y;
         } else {
-          hi[s][T][h][0] = 0; hi[s][T][h][1] = 0;
+          hi[T][h][0] = 0; hi[T][h][1] = 0;
         }
       }
     }
-  }
-#pragma unroll
-  for (int s = 0; s < NSUB; ++s)
-    chunk_mmas<R, NT, TW>(lo[s], hi[s], xaddr, xstep, s * G::W8, cd, errp, ch,
+    chunk_mmas<R, NT, TW>(lo, hi, xaddr, xstep, s * G::W8, cd, rs, errp, ch,
                           std::make_integer_sequence<int, G::W8>{});
+  }
 }
 
 // The current linear of a CTA's walk over its unit range, cached in registers.
@@ -460,24 +506,27 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
 }
 
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
-// removes the decoding offsets and the zero point (once per row, by the part
-// that starts at k-chunk 0) and writes y. A row block this CTA owns whole is
-// stored; a shared one is added atomically into y, which the prep kernel
-// zeroed.
+// removes the zero point (once per row, by the part that starts at k-chunk 0)
+// and writes y. The bf16 decode sums x (c - c0), so its zero point is taken
+// relative to the row's centre code: y = A acc - alpha (z - c0 2^(8-r)) Sx;
+// the integer kinds sum x c: y = A acc - alpha z Sx. A row block this CTA
+// owns whole is stored; a shared one is added atomically into y, which the
+// prep kernel zeroed.
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
                            int T, int lane, const float (&tot)[NT][4]) {
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
-  float c[kClasses];
-  offset_coeffs(L.dk, L.r, c);
+  const int cmax = L.dk == 11 ? (1 << L.r) : (1 << L.r) - 1;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h;
     if (n >= L.N) continue;
     const float a = L.alpha[n], z = L.zero[n];
-    const float A = a * scale, B = a * z;
+    // the same centre code the decode subtracted (make_rowsub)
+    const float c0 = is_i8(L.dk) ? 0.f : static_cast<float>(centre_code(z, L.r, cmax));
+    const float A = a * scale, B = a * (z - c0 * scale);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -489,13 +538,10 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
           // Extra Precision: each listed position adds one code step
           if (L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
           const float* P = L.psum + m * kClasses;
-          float O = 0.f, Sx = 0.f;
+          float Sx = 0.f;
 #pragma unroll
-          for (int i = 0; i < kClasses; ++i) {
-            O = fmaf(c[i], P[i], O);
-            Sx += P[i];
-          }
-          v = A * (v - O) - B * Sx;
+          for (int i = 0; i < kClasses; ++i) Sx += P[i];
+          v = A * v - B * Sx;
         } else {
           v = A * v;
         }
@@ -517,8 +563,20 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
                                             volatile int* s_abort, int seg, int& s, uint32_t& ph,
                                             bool active, const uint32_t (&xaddr)[NT],
                                             const uint32_t (&xstep)[NT], int warp, int lane,
-                                            const Cdec& cd, float (&tot)[Tiling<NT>::TW][NT][4]) {
+                                            const Cdec& cd, int l, int rb,
+                                            float (&tot)[Tiling<NT>::TW][NT][4]) {
   constexpr int TW = Tiling<NT>::TW;
+  // the centre codes of this thread's rows (rows g and g + 8 of each tile)
+  RowSub rs[TW][2];
+  {
+    const LinDesc& L = p.lin[l];
+    const int g = lane >> 2;
+#pragma unroll
+    for (int T = 0; T < TW; ++T)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h, L.N, L.r);
+  }
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
       if (lane == 0) { atomicOr(p.err, kErrWaitFull); *s_abort = 1; }
@@ -539,7 +597,7 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
 #pragma unroll
           for (int j = 0; j < 4; ++j) { ch[T][b][0][j] = 0.f; ch[T][b][1][j] = 0.f; }
       // the plane pitches and rows follow from the batch tiles (Tiling)
-      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, cd, p.err, ch);
+      process_unit<R, NT>(st, st + Tiling<NT>::RPU * Tiling<NT>::P0, xa, xstep, warp, lane, cd, rs, p.err, ch);
 #pragma unroll
       for (int T = 0; T < TW; ++T)
 #pragma unroll
@@ -640,14 +698,15 @@ __device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xad
 // digits cannot hold exactly, the bf16 fragments of the width's bf16 path
 // (mode 1). Thread (g, t) of a digit unit holds the int32 sums of columns 2t
 // and 2t + 1, digits 2t and 2t + 1 (column 7 is zero): it weighs them by
-// 2^(7 digit - sigma), sigma = 48 - E. A bf16 unit's offset sum is taken out by
-// thread t = 0. The partials stay in tot[T][0][0] (row g) and tot[T][0][2]
-// (row g + 8) until the row block is flushed.
+// 2^(7 digit - sigma), sigma = 48 - E. A bf16 unit sums x (c - c0) per row;
+// thread t = 0 adds c0 Sxu back (Sxu, the unit's input sum, is in the
+// header). The partials stay in tot[T][0][0] (row g) and tot[T][0][2] (row
+// g + 8) until the row block is flushed.
 template <int R, int CAP>
 __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const uint8_t* stages,
                                                uint64_t* full, uint64_t* empty, volatile int* s_abort,
                                                int seg, int& s, uint32_t& ph, bool active,
-                                               uint32_t zero_addr, int warp, int lane,
+                                               uint32_t zero_addr, int warp, int lane, int l, int rb,
                                                float (&tot)[2][1][4]) {
   const int g = lane >> 2, t = lane & 3;
   for (int i = 0; i < seg; ++i) {
@@ -682,8 +741,10 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
                               fmaf(static_cast<float>(ch[T][0][3] + ch[T][1][3]), w1, tot[T][0][2]));
         }
       } else {
-        // bf16 fragments of batch row 0 (lanes g = 0), the width's bf16 decode
-        const float O = t == 0 ? reinterpret_cast<const float*>(hdr)[2] : 0.f;
+        // bf16 fragments of batch row 0 (lanes g = 0), the width's bf16 decode,
+        // which sums x (c - c0): thread t = 0 adds c0 Sxu back (Sxu = the
+        // unit's input sum from the header)
+        const float Sxu = t == 0 ? reinterpret_cast<const float*>(hdr)[2] : 0.f;
         float ch[2][1][2][4];
 #pragma unroll
         for (int T = 0; T < 2; ++T)
@@ -691,12 +752,21 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
           for (int j = 0; j < 4; ++j) { ch[T][0][0][j] = 0.f; ch[T][0][1][j] = 0.f; }
         const uint32_t xa[1] = {g == 0 ? xs + static_cast<uint32_t>(t) * 16u : zero_addr};
         const uint32_t xstep[1] = {g == 0 ? 64u : 0u};
+        // the centre codes of this thread's rows, made here (a rare path)
+        // rather than held in registers across the unit loop
+        RowSub rs[2][2];
+        const LinDesc& L = p.lin[l];
+#pragma unroll
+        for (int T = 0; T < 2; ++T)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<1>::RPU + warp * Tiling<1>::RPW + 16 * T + g + 8 * h, L.N, L.r);
         process_unit<R, 1>(st, st + Tiling<1>::RPU * Tiling<1>::P0, xa, xstep, warp, lane, Cdec{0u, 0u, 0u},
-                           p.err, ch);
+                           rs, p.err, ch);
 #pragma unroll
         for (int T = 0; T < 2; ++T) {
-          tot[T][0][0] += (ch[T][0][0][0] + ch[T][0][1][0]) - O;
-          tot[T][0][2] += (ch[T][0][0][2] + ch[T][0][1][2]) - O;
+          tot[T][0][0] += fmaf(rs[T][0].c0, Sxu, ch[T][0][0][0] + ch[T][0][1][0]);
+          tot[T][0][2] += fmaf(rs[T][1].c0, Sxu, ch[T][0][0][2] + ch[T][0][1][2]);
         }
       }
     }
@@ -707,7 +777,10 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
   return true;
 }
 
-template <int NT, int CAP>
+// I8: a launch whose linears all take the integer kinds (one batch row,
+// planes of width 8, 4, 2): its instantiation holds only their code paths, so
+// the registers of the bf16 decodes do not press on the integer loop.
+template <int NT, int CAP, bool I8 = false>
 __global__ void __launch_bounds__(kGemvThreads, (NT <= 2 ? 2 : 1))
 gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   using TL = Tiling<NT>;
@@ -838,27 +911,35 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         for (int i = 0; i < 4; ++i) tot[T][b][i] = 0.f;
     bool ok;
     const Cdec cd = make_cdec(c.dk, c.r);
-    switch (c.dk) {
-      case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
-      // the host plans the integer kinds only for one batch row
-      case kDkI8 + 8:
-        if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
-        else ok = false;
-        break;
-      case kDkI8 + 4:
-        if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
-        else ok = false;
-        break;
-      case kDkI8 + 2:
-        if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, tot);
-        else ok = false;
-        break;
-      default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, tot); break;
+    if constexpr (I8) {
+      switch (c.dk) {
+        case kDkI8 + 8: ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
+        case kDkI8 + 4: ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
+        default: ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
+      }
+    } else {
+      switch (c.dk) {
+        case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        // the host plans the integer kinds only for one batch row
+        case kDkI8 + 8:
+          if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          else ok = false;
+          break;
+        case kDkI8 + 4:
+          if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          else ok = false;
+          break;
+        case kDkI8 + 2:
+          if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          else ok = false;
+          break;
+        default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+      }
     }
     if (!ok) break;  // outputs are undefined after a give-up; the flag says so
     if (active) {
@@ -1014,7 +1095,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
   // biased exponent e, -133 for a subnormal) becomes X = m 2^(f + 48 - E),
   // below 2^49, an integer when f >= E - 48; digit g is (X >> 7g) & 127 with
   // x's sign. A unit with f < E - 48 somewhere, a non-finite input or E
-  // outside [-78, 100] gets the width's bf16 fragments and offset sum instead
+  // outside [-78, 100] gets the width's bf16 fragments and input sum instead
   // (written by the digit-0 warp).
   if (p.n_i8 > 0) {
     const int lane = threadIdx.x & 31;
@@ -1131,14 +1212,8 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
           if (kg < L.K) v = *reinterpret_cast<const uint4*>(xr + kg);
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float xv = __uint_as_float(((u & 1) ? (w4[u >> 1] >> 16) : (w4[u >> 1] & 0xFFFFu)) << 16);
-            // the bf16 path's magic offset of input kg + u: 16 at r = 4, the
-            // class magics (k >> 1) & 7 at r = 2, none at r = 8 (kg % 8 == 0)
-            constexpr float kMagic2[kClasses] = {64.f, 16.f, 4.f, 64.f, 16.f, 4.f, 64.f, 16.f};
-            const float off = r == 4 ? 16.f : r == 2 ? kMagic2[((kg + u) >> 1) & 7] : 0.f;
-            part = fmaf(xv, off, part);
-          }
+          for (int u = 0; u < 8; ++u)  // the unit's input sum: the fold adds c0 times it back
+            part += __uint_as_float(((u & 1) ? (w4[u >> 1] >> 16) : (w4[u >> 1] & 0xFFFFu)) << 16);
           if (r == 8) {
             const uint32_t a = __byte_perm(v.x, v.y, 0x5410), b = __byte_perm(v.x, v.y, 0x7632);
             const uint32_t c = __byte_perm(v.z, v.w, 0x5410), d = __byte_perm(v.z, v.w, 0x7632);
@@ -1210,9 +1285,9 @@ std::mutex g_cache_mutex;
 
 // Persistent grid for `units` work units at `smem` bytes of shared memory:
 // every resident CTA slot of the device, at most one CTA per unit.
-template <int NT, int CAP>
+template <int NT, int CAP, bool I8 = false>
 cudaError_t gemv_grid(size_t smem, int sms, int units, int* grid_out) {
-  auto kern = gemv_streamk_kernel<NT, CAP>;
+  auto kern = gemv_streamk_kernel<NT, CAP, I8>;
   static std::map<int, KernelCache> caches;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1240,9 +1315,9 @@ cudaError_t gemv_grid(size_t smem, int sms, int units, int* grid_out) {
   return cudaSuccess;
 }
 
-template <int NT, int CAP>
+template <int NT, int CAP, bool I8 = false>
 cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int grid, cudaStream_t stream) {
-  auto kern = gemv_streamk_kernel<NT, CAP>;
+  auto kern = gemv_streamk_kernel<NT, CAP, I8>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -1459,9 +1534,11 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   stages = std::max(2, std::min(stages, kMaxStages));
   const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(stages) * stage_bytes;
   const int sms = sm_count();
+  bool i8_only = true;
+  for (int i = 0; i < n_jobs; ++i) i8_only = i8_only && is_i8(gp.lin[i].dk);
   int grid = 1;
   switch (NT) {
-    case 1: e = gemv_grid<1, CAP>(smem, sms, units, &grid); break;
+    case 1: e = i8_only ? gemv_grid<1, CAP, true>(smem, sms, units, &grid) : gemv_grid<1, CAP>(smem, sms, units, &grid); break;
     case 2: e = gemv_grid<2, CAP>(smem, sms, units, &grid); break;
     case 3: e = gemv_grid<3, CAP>(smem, sms, units, &grid); break;
     default: e = gemv_grid<4, CAP>(smem, sms, units, &grid); break;
@@ -1556,7 +1633,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.wait_ns = wait_limit_ns();
 
   switch (NT) {
-    case 1: return launch_gemv<1, CAP>(gp, smem, grid, stream);
+    case 1: return i8_only ? launch_gemv<1, CAP, true>(gp, smem, grid, stream) : launch_gemv<1, CAP>(gp, smem, grid, stream);
     case 2: return launch_gemv<2, CAP>(gp, smem, grid, stream);
     case 3: return launch_gemv<3, CAP>(gp, smem, grid, stream);
     default: return launch_gemv<4, CAP>(gp, smem, grid, stream);

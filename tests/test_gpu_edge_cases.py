@@ -7,9 +7,9 @@ GEMM above), within |y - y_ref| <= 1e-3 sum_k |x||W_r| + 1e-6:
   with nonzero inputs;
 * constant rows (max = min): alpha = max(|min| 2^-8, 2^-126), z = -min /
   alpha, every code 0, and W_r = min exactly, so y = min * sum_k x;
-* rows whose zero point sits exactly on a code level: most weights dequantize
-  to exactly 0 at every width, so the bound shrinks towards 1e-6 while the
-  kernels form y = A (acc - O) - B Sx from large terms.
+* rows whose zero point sits exactly on a code level (the centre code or
+  another): most weights dequantize to exactly 0 at every width, so the bound
+  shrinks towards 1e-6 while the kernels form y from sums of codes and of x.
 """
 import numpy as np
 import pytest
@@ -86,39 +86,39 @@ def test_constant_rows(r, m):
         assert np.all(np.abs(y[:, i] - ref) <= tol)
 
 
-def _zero_on_code_level(n, k, density, seed):
-    """Rows with min = -1 and max = 127/128 (alpha = 2^-7, z = 128, a code
-    level at every width: S(128, r) = 128), the rest 0 except a `density`
-    fraction of uniform weights in [-1, 0.98] rounded to bf16."""
+def _zero_on_code_level(n, k, density, seed, zlevel):
+    """Rows with min = -zlevel 2^-7 and max = (255 - zlevel) 2^-7, so alpha =
+    2^-7 and z = zlevel exactly, a code level at every width for zlevel = 128
+    (the centre) and 64; the rest 0 except a `density` fraction of uniform
+    weights inside the range, rounded to bf16."""
     rng = np.random.default_rng(seed)
+    lo, hi = -zlevel / 128.0, (255 - zlevel) / 128.0
     w = np.zeros((n, k), dtype=np.float32)
     mask = rng.random((n, k)) < density
-    w[mask] = rng.uniform(-1.0, 0.98, size=int(mask.sum()))
+    w[mask] = rng.uniform(lo, 0.98 * hi, size=int(mask.sum()))
     cols = rng.integers(0, k, size=(n, 2))
     cols[:, 1] = (cols[:, 0] + 1 + cols[:, 1] % (k - 1)) % k
-    w[np.arange(n), cols[:, 0]] = -1.0
-    w[np.arange(n), cols[:, 1]] = 127.0 / 128.0
+    w[np.arange(n), cols[:, 0]] = lo
+    w[np.arange(n), cols[:, 1]] = hi
     return synth.bf16_bits_from_f32(w)
 
 
-# The paths whose accumulation is exact in integers (one batch row, r = 8, 4,
-# 2) keep this case within the bound; the bf16 paths carry each code's magic
-# offset through fp32 sums and do not yet.
-@pytest.mark.parametrize("r", [8, 4, 2])
-@pytest.mark.parametrize("m", [1])
-@pytest.mark.parametrize("k,density", [(4096, 0.0), (4096, 0.01), (14336, 0.002)])
-def test_zero_point_on_a_code_level(r, m, k, density):
+@pytest.mark.parametrize("r", WIDTHS)
+@pytest.mark.parametrize("m", [1, 2, 8, 32, 64])
+@pytest.mark.parametrize("k,density,zlevel", [(4096, 0.0, 128), (4096, 0.01, 128), (14336, 0.002, 128),
+                                              (4096, 0.0, 64), (14336, 0.002, 64)])
+def test_zero_point_on_a_code_level(r, m, k, density, zlevel):
     n = 256
-    w_bits = _zero_on_code_level(n, k, density, 17 + k + m)
+    w_bits = _zero_on_code_level(n, k, density, 17 + k + m, zlevel)
     w_vals = synth.f32_from_bf16_bits(w_bits).astype(np.float64)
     q_d, a_d, z_d = gpu_quantize(w_bits, "bf16")
     q, a, z = oracle.quantize_minmax(w_vals)
-    assert np.all(a == 2.0 ** -7) and np.all(z == 128.0)
+    assert np.all(a == 2.0 ** -7) and np.all(z == float(zlevel))
     assert np.array_equal(q_d.cpu().numpy(), q)
     wr = oracle.dequant_slice(q, a, z, r)
     assert (wr == 0.0).mean() > 0.95
     x_bits = synth.activations(m, k, 970 + m)
     x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
     y = _linear(x_bits, gpu_pack(q_d, r), a_d, z_d, n, r)
-    ratio = check_linear(y, x_vals, wr, f"z on a code level r={r} M={m} K={k} density={density}")
-    print(f"r={r} M={m} K={k} density={density}: worst err/tol {ratio:.3f}")
+    ratio = check_linear(y, x_vals, wr, f"z on a code level r={r} M={m} K={k} density={density} z={zlevel}")
+    print(f"r={r} M={m} K={k} density={density} z={zlevel}: worst err/tol {ratio:.3f}")
