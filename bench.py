@@ -206,6 +206,19 @@ class Stack:
         lol = [remap[self.lol[i]] for i in idx]
         return lins, lol, [width] * len(layers), len(layers)
 
+    def with_batch(self, M: int):
+        """The stack's packed weights with inputs and outputs for batch M (the
+        weights are not rebuilt): (lins, y buffer)."""
+        import torch
+        xs = {k: synth.device_activations(M, k, 2000 + M + k, self.dev) for k in self.Ks}
+        n_out = sum(n for (_, _, _, _, _, n, _) in self.lins)
+        y_all = torch.empty(M * n_out, dtype=torch.float32, device=self.dev)
+        out, off = [], 0
+        for (_, p, a, z, _, n, k) in self.lins:
+            out.append((xs[k], p, a, z, y_all[off:off + M * n].view(M, n), n, k))
+            off += M * n
+        return out, y_all
+
     def lins_with_y(self, y_all):
         """The stack's linears with their outputs in another buffer of y_all's shape."""
         out, off = [], 0
@@ -370,6 +383,144 @@ def rows_timings(dev, stream):
     return out
 
 
+def configs_timings(dev, stream, stack, hbm_peak, steps):
+    """The per-configuration decode numbers, each on its own shapes and laws:
+    single linear (512 x 1024 fp32 weights, r = 8, 4, 2, M = 1); a Gemma-2-2B
+    decode layer (q, k, v, o 2304 x 2304, gate, up 9216 x 2304, down
+    2304 x 9216) at r = 4, M = 1, 4, 8, one grouped launch per layer; the
+    Mistral-7B MLP (14336 x 4096 and 4096 x 14336, Student-t(4) * 0.02) at
+    r = 2, 4, 8 and M = 1, 4, 16, 32, one launch per MLP; and the 7B
+    Mix'n'Match stack at M = 2, 4, 8, 16, 32. The small configurations fit in
+    L2, so each is timed round robin over enough copies of its weights
+    (packed planes, alpha, z) to span at least 4x L2; every time is device time
+    (CUDA events) per call, after warm-up."""
+    import torch
+    import nested_bit_weight_int8_b200 as mq
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", L2_BYTES)
+
+    def quantized(w_dev, dtype_code, n, k):
+        q = torch.empty((n, k), dtype=torch.uint8, device=dev)
+        a = torch.empty(n, dtype=torch.float32, device=dev)
+        z = torch.empty(n, dtype=torch.float32, device=dev)
+        mq.quantize_int8(w_dev, dtype_code, n, k, q, a, z, stream)
+        return q, a, z
+
+    def copies(packed_bytes):
+        return max(4, int(4 * l2 // max(1, packed_bytes)) + 1)
+
+    def time_round_robin(plans, reps):
+        """Device time per call of one pass over `plans`, replayed from a CUDA
+        graph (launched directly, the host's enqueue rate would set the pace
+        of such short calls)."""
+        for _ in range(2):
+            for pl in plans:
+                pl.run(stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for pl in plans:
+                pl.run(stream)
+        graph.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del graph
+        return e0.elapsed_time(e1) * 1000.0 / (reps * len(plans))  # us per call
+
+    def entry(us, packed, M):
+        gbs = packed / (us * 1e-6) / 1e9
+        return {"us": round(us, 2), "GBps": round(gbs, 1), "frac_of_hbm": round(gbs / hbm_peak, 3),
+                "tokens_per_s": round(M / (us * 1e-6), 1)}
+
+    out = {}
+    # config 1: one 512 x 1024 linear, fp32 weights N(0, 0.02^2), seed 0
+    n, k = 512, 1024
+    w = torch.from_numpy(synth.gaussian_weights(n, k, 0, dtype="f32")).to(dev)
+    q, a, z = quantized(w, mq.MQ_F32, n, k)
+    x = torch.from_numpy(synth.activations(1, k, 1).view(np.int16)).to(dev)
+    c1 = {}
+    for r in (8, 4, 2):
+        nb = n * k * r // 8
+        lins = []
+        for _ in range(copies(nb)):
+            p = torch.empty(mq.packed_bytes(n, k, r), dtype=torch.uint8, device=dev)
+            mq.slice_pack(q, n, k, r, p, stream)
+            lins.append(mq.StackPlan([(x, p, a.clone(), z.clone(), torch.empty((1, n), dtype=torch.float32, device=dev), n, k)],
+                                     [0], [r], 1))
+        c1[f"r{r}_M1"] = entry(time_round_robin(lins, 3), nb, 1)
+    out["single_linear_512x1024_f32"] = c1
+    del w, q, lins
+    # config 2: a Gemma-2-2B decode layer at r = 4, one grouped launch
+    mats = synth.WORKLOADS["gemma2_2b_decode_layer"]["mats"]
+    base = []
+    for i, (_, n, k) in enumerate(mats):
+        w = synth.device_gaussian_weights(n, k, 100 + i, dev)
+        q, a, z = quantized(w, mq.MQ_BF16, n, k)
+        p = torch.empty(mq.packed_bytes(n, k, 4), dtype=torch.uint8, device=dev)
+        mq.slice_pack(q, n, k, 4, p, stream)
+        base.append((p, a, z, n, k))
+        del w, q
+    layer_bytes = sum(n * k * 4 // 8 for (_, _, _, n, k) in base)
+    c2 = {}
+    n_copies = copies(layer_bytes)
+    layers = [[(p.clone(), a.clone(), z.clone(), n, k) for (p, a, z, n, k) in base] for _ in range(n_copies)]
+    for M in (1, 4, 8):
+        xs = {k: synth.device_activations(M, k, 200 + M + k, dev) for k in {k for (*_, k) in base}}
+        plans = []
+        for lay in layers:
+            lins = [(xs[k], p, a, z, torch.empty((M, n), dtype=torch.float32, device=dev), n, k)
+                    for (p, a, z, n, k) in lay]
+            plans.append(mq.StackPlan(lins, [0] * len(lins), [4], M))
+        c2[f"r4_M{M}"] = entry(time_round_robin(plans, 3), layer_bytes, M)
+    c2["per"] = "layer (7 linears, one launch)"
+    out["gemma2_2b_layer_r4"] = c2
+    del layers, base
+    # config 3: the Mistral-7B MLP, heavy-tailed weights, r = 2, 4, 8
+    mats = synth.WORKLOADS["mistral7b_mlp_heavy_tail"]["mats"]
+    qs = []
+    for i, (_, n, k) in enumerate(mats):
+        w = torch.from_numpy(synth.student_t_weights(n, k, 300 + i).view(np.int16)).to(dev)
+        qs.append((*quantized(w, mq.MQ_BF16, n, k), n, k))
+        del w
+    c3 = {}
+    for r in (2, 4, 8):
+        mlp_bytes = sum(n * k * r // 8 for (*_, n, k) in qs)
+        n_copies = copies(mlp_bytes)
+        packs = []
+        for (q, a, z, n, k) in qs:
+            p = torch.empty(mq.packed_bytes(n, k, r), dtype=torch.uint8, device=dev)
+            mq.slice_pack(q, n, k, r, p, stream)
+            packs.append((p, a, z, n, k))
+        mlps = [[(p.clone(), a.clone(), z.clone(), n, k) for (p, a, z, n, k) in packs] for _ in range(n_copies)]
+        for M in (1, 4, 16, 32):
+            xs = {k: synth.device_activations(M, k, 400 + M + k, dev) for k in {k for (*_, k) in qs}}
+            plans = [mq.StackPlan([(xs[k], p, a, z, torch.empty((M, n), dtype=torch.float32, device=dev), n, k)
+                                   for (p, a, z, n, k) in mlp], [0, 0], [r], M) for mlp in mlps]
+            c3[f"r{r}_M{M}"] = entry(time_round_robin(plans, 3), mlp_bytes, M)
+        del mlps, packs
+    c3["per"] = "MLP (up 14336x4096 + down 4096x14336, one launch)"
+    out["mistral7b_mlp_student_t"] = c3
+    del qs
+    # config 4 at larger batches: the same packed stack, new inputs per M
+    c4 = {}
+    for M in (2, 4, 8, 16, 32):
+        lins, y_all = stack.with_batch(M)
+        plan = mq.StackPlan(lins, stack.lol, stack.widths, M)
+        ms = time_device(lambda: plan.run(stream), max(3, steps // 8), 3, stream, 1, dev)
+        c4[f"M{M}"] = entry(ms * 1000.0, stack.packed_bytes, M)
+        c4[f"M{M}"]["us_per_layer"] = round(ms * 1000.0 / stack.layers, 2)
+        del lins, y_all, plan
+    c4["per"] = "step (32 layers, 160 linears, one launch)"
+    out["mixnmatch_7b_stack_batches"] = c4
+    torch.cuda.synchronize()
+    return out
+
+
 def cpu_baseline(M: int, budget_s: float = 12.0):
     """The CPU oracle (float64 numpy) on a bounded sample of the same
     workload: dequantize-and-multiply for row blocks of the stack's linears,
@@ -505,12 +656,18 @@ def run_gpu(args, rank, world, local):
         ms_e2e = time_device(e2e_step, max(3, args.steps // 4), 3, stream, world, dev, finish=e2e_finish)
 
         rows = rows_timings(dev, stream) if rank == 0 and not args.no_rows else {}
+        configs = (configs_timings(dev, stream, stack, hbm_peak, args.steps)
+                   if rank == 0 and not args.no_configs and WORKLOAD == "mixnmatch_7b_stack"
+                   and len(stack.lins) == 160 and args.M == 1 else {})
     torch.cuda.synchronize()
 
     gbs = stack.packed_bytes / (ms * 1e-3) / 1e9
     algo = stack.algorithmic_bytes()
     achieved = algo / (ms * 1e-3) / 1e9
+    # The driver keeps the tail of the printed line, so the long "rows" block
+    # comes first and the per-width and per-configuration numbers last.
     out = {
+        "rows": rows,
         "metric": METRIC,
         "value": round(gbs * world, 1),
         "unit": "GB/s",
@@ -538,7 +695,6 @@ def run_gpu(args, rank, world, local):
         "pct_of_hbm_peak": round(100 * gbs / hbm_peak, 1),
         "us_per_layer": round(ms * 1000 / stack.layers, 2),
         "tokens_per_s": round(args.M * world * 1000.0 / ms, 1),
-        "per_width": per_width,
         "chain": chain,
         "roofline": {
             "bound": "hbm",
@@ -561,11 +717,12 @@ def run_gpu(args, rank, world, local):
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
-        "rows": rows,
     }
     tr = _profile_traffic()
     if tr is not None and tr.get("kernel_source_hash") == _kernel_hash():
         out["roofline"]["traffic"] = tr.get("dram_bytes_per_launch")
+    out["configs"] = configs
+    out["per_width"] = per_width
     return out
 
 
@@ -664,6 +821,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-chain", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration decode timings (configs 1-3, stack at M = 2..32)")
     ap.add_argument("--results", default="",
                     help="also append each JSON line, time-stamped, to this JSON-lines file")
     ap.add_argument("--no-cpu", action="store_true")
@@ -693,7 +852,11 @@ def main(argv=None):
         out = run_gpu(args, rank, world, local)
         if rank == 0:
             if not args.no_cpu:
-                out["cpu_baseline"] = cpu_baseline(args.M)
+                # before the per-width and per-configuration blocks, which stay last
+                cb = cpu_baseline(args.M)
+                tail = {key: out.pop(key) for key in ("configs", "per_width")}
+                out["cpu_baseline"] = cb
+                out.update(tail)
             emit(out, args.results)
         return 0
     finally:

@@ -89,10 +89,11 @@ constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
 // codes). Its staged activation block is a 64-byte header (int mode: 0 digits,
 // 1 bf16 fragments; int E, the unit's largest exponent; float Sxu, the input
 // sum of a bf16 unit) and then slot (s, jj, t, g) of 16 bytes at
-// 64 + (((s * J / 2 + jj) * 4 + t) * kI8Digits + g) * 16, J = 16 / r MMAs per
+// 64 + (((s * J / 2 + jj) * kI8Digits + g) * 4 + t) * 16, J = 16 / r MMAs per
 // 16-byte chunk: digit g of the 16 inputs of MMAs 2 jj and 2 jj + 1 of chunk
-// 4s + t, in their k-slot order (b0, b1 of each). A mode-1 unit holds the
-// width's bf16 fragments there instead.
+// 4s + t, in their k-slot order (b0, b1 of each); lane 4g + t reads slot
+// (g, t), so each 8-lane phase of the 16-byte load reads 128 contiguous bytes.
+// A mode-1 unit holds the width's bf16 fragments there instead.
 constexpr int kDkI8 = 20;
 constexpr int kI8Digits = 7;
 constexpr int kI8Header = 64;
@@ -115,6 +116,11 @@ struct Tiling {
   static constexpr int P0 = (NT == 1) ? 128 : 64;    // plane-0 bytes per row per unit
   static constexpr bool SWZ = (NT == 1);             // plane-0 box in 128-byte swizzle
   static constexpr int NSUB = P0 / 64;               // 64-byte sub-steps per unit
+  // Unit row (within a 16-row tile, before + 8h) of MMA fragment row g. With
+  // the 128-byte swizzle (chunk c of row w at c ^ (w % 8)) the two rows that
+  // one 8-lane phase of a 16-byte load reads (g = 2p, 2p + 1) are made to
+  // differ in bit 2, which puts their chunks in different bank groups.
+  static __device__ __forceinline__ int frag_row(int g) { return SWZ ? (((g & 1) << 2) | (g >> 1)) : g; }
 };
 // The same choice on the host, by batch size.
 inline int tiling_p0(int M) { return M <= 8 ? 128 : 64; }
@@ -448,7 +454,7 @@ __device__ __forceinline__ void process_unit(const uint8_t* st0, const uint8_t* 
     for (int T = 0; T < TW; ++T) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int row = warp * TL::RPW + 16 * T + g + 8 * h;
+        const int row = warp * TL::RPW + 16 * T + TL::frag_row(g) + 8 * h;
         const int cs = TL::SWZ ? (ci ^ (row & 7)) : ci;
         const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * P0 + cs * 16);
         lo[T][h][0] = v.x; lo[T][h][1] = v.y; lo[T][h][2] = v.z; lo[T][h][3] = v.w;
@@ -521,7 +527,7 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
   const int cmax = L.dk == 11 ? (1 << L.r) : (1 << L.r) - 1;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h;
+    const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
     if (n >= L.N) continue;
     const float a = L.alpha[n], z = L.zero[n];
     // the same centre code the decode subtracted (make_rowsub)
@@ -575,7 +581,7 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
     for (int T = 0; T < TW; ++T)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + g + 8 * h, L.N, L.r);
+        rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h, L.N, L.r);
   }
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
@@ -680,7 +686,7 @@ __device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xad
     for (int T = 0; T < TW; ++T) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int row = warp * TL::RPW + 16 * T + g + 8 * h;
+        const int row = warp * TL::RPW + 16 * T + TL::frag_row(g) + 8 * h;
         const int cs = ci ^ (row & 7);  // 128-byte swizzle
         const uint4 v = *reinterpret_cast<const uint4*>(st0 + row * P0 + cs * 16);
         lo[s][T][h][0] = v.x; lo[s][T][h][1] = v.y; lo[s][T][h][2] = v.z; lo[s][T][h][3] = v.w;
@@ -728,7 +734,7 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
 #pragma unroll
           for (int j = 0; j < 4; ++j) { ch[T][0][j] = 0; ch[T][1][j] = 0; }
         const bool live = g < kI8Digits;
-        process_unit_i8<R>(st, live ? xs + static_cast<uint32_t>(t * kI8Digits + g) * 16u : zero_addr,
+        process_unit_i8<R>(st, live ? xs + static_cast<uint32_t>(g * 4 + t) * 16u : zero_addr,
                            live ? 4u * kI8Digits * 16u : 0u, warp, lane, p.err, ch);
         // digit 2t weighs 2^(14t + E - 48), digit 2t + 1 2^(14t + 7 + E - 48)
         const float w0 = __int_as_float((127 + 14 * t + E - 48) << 23);
@@ -760,7 +766,7 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
         for (int T = 0; T < 2; ++T)
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<1>::RPU + warp * Tiling<1>::RPW + 16 * T + g + 8 * h, L.N, L.r);
+            rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<1>::RPU + warp * Tiling<1>::RPW + 16 * T + Tiling<1>::frag_row(g) + 8 * h, L.N, L.r);
         process_unit<R, 1>(st, st + Tiling<1>::RPU * Tiling<1>::P0, xa, xstep, warp, lane, Cdec{0u, 0u, 0u},
                            rs, p.err, ch);
 #pragma unroll
@@ -1034,12 +1040,22 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
     // 8 consecutive elements k0..k0+7 (k0 % 8 == 0) fall in classes
     // 4h, 4h, 4h+1, 4h+1, ..., 4h+3 with h = (k0 >> 3) & 1; the stride of
     // the loop is a multiple of 16, so h is the parity of the thread.
-    for (int k0 = threadIdx.x * 8; k0 < J.K; k0 += blockDim.x * 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(row + k0);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    // eight loads in flight per thread before any add (the row is read once,
+    // from L2 or HBM, and this CTA is on the decode kernel's critical path)
+    for (int kb = threadIdx.x * 8; kb < J.K; kb += blockDim.x * 64) {
+      uint4 u[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        acc[i] += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
+      for (int j = 0; j < 8; ++j) {
+        const int k0 = kb + j * blockDim.x * 8;
+        u[j] = k0 < J.K ? *reinterpret_cast<const uint4*>(row + k0) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          acc[i] += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     }
     __shared__ float red[kClasses][8];
 #pragma unroll
@@ -1191,7 +1207,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
             const uint32_t sd = (bits & 0x8000u) ? (0u - d) & 0xFFu : d;
             out[b >> 2] |= sd << (8 * (b & 3));
           }
-          const int64_t off = kI8Header + (int64_t((s * J2 + jj) * 4 + t) * kI8Digits + g) * 16;
+          const int64_t off = kI8Header + (int64_t((s * J2 + jj) * kI8Digits + g) * 4 + t) * 16;
           if (MQ_IN_BOUNDS(int64_t(kc) * i8_unit_bytes(r) + off + 16 <= blk_end, p.err))
             *reinterpret_cast<uint4*>(blk + off) = make_uint4(out[0], out[1], out[2], out[3]);
         }
