@@ -156,6 +156,10 @@ struct GemvParams {
   int pitch0, pitch1;
   uint32_t* err;
   unsigned long long wait_ns;
+  // 4, 16, 64: left shifts of the integer decode done as multiplies (the FMA
+  // pipe) instead of shifts (the ALU pipe, its busiest); as kernel
+  // parameters the compiler cannot turn them back into shifts
+  uint32_t shl[3];
   int cta_begin[kMaxCtas + 1];  // unit range of CTA c: [cta_begin[c], cta_begin[c + 1])
   LinDesc lin[CAP];
 };
@@ -620,26 +624,35 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
 
 // The A registers of MMA j of a 16-byte chunk for one weight row (words
 // w[0..3] of the chunk) on the integer path: codes as bytes, in k-slot order
-// k 4t + i (a0) and 16 + 4t + i (a2).
+// k 4t + i (a0) and 16 + 4t + i (a2), each code in the top bits of its byte
+// (a power-of-two multiple, taken out when the unit is folded).
 //  r = 8: the bytes themselves; a0 = word 2j, a2 = word 2j + 1.
-//  r = 4: word j holds codes u at bit 16 (u % 2) + 4 (u / 2); w & 0x0F0F0F0F
-//         gives codes 0, 4, 1, 5 and (w >> 4) & 0x0F0F0F0F codes 2, 6, 3, 7.
+//  r = 4: word j holds codes u at bit 16 (u % 2) + 4 (u / 2);
+//         (w << 4) & 0xF0F0F0F0 gives 16 x codes 0, 4, 1, 5 and
+//         w & 0xF0F0F0F0 16 x codes 2, 6, 3, 7.
 //  r = 2: word j / 2 holds 16 codes at bit 16 (u % 2) + 2 (u / 2);
-//         (w >> 2i) & 0x03030303 gives codes 2i, 2i + 8, 2i + 1, 2i + 9, and
-//         MMA j takes i = 2 (j % 2) (a0) and i = 2 (j % 2) + 1 (a2).
+//         (w << (6 - 2i)) & 0xC0C0C0C0 gives 64 x codes 2i, 2i + 8, 2i + 1,
+//         2i + 9, and MMA j takes i = 2 (j % 2) (a0) and i = 2 (j % 2) + 1 (a2).
+// The left shifts are multiplies by the kernel parameters shl = {4, 16, 64}.
 template <int R, int J>
-__device__ __forceinline__ void i8_regs(const uint32_t (&w)[4], uint32_t& a0, uint32_t& a2) {
+__device__ __forceinline__ void i8_regs(const uint32_t (&w)[4], const uint32_t (&shl)[3], uint32_t& a0,
+                                        uint32_t& a2) {
   if constexpr (R == 8) {
     a0 = w[2 * J];
     a2 = w[2 * J + 1];
   } else if constexpr (R == 4) {
-    a0 = w[J] & 0x0F0F0F0Fu;
-    a2 = (w[J] >> 4) & 0x0F0F0F0Fu;
+    a0 = (w[J] * shl[1]) & 0xF0F0F0F0u;
+    a2 = w[J] & 0xF0F0F0F0u;
+  } else if constexpr (J % 2 == 0) {
+    a0 = (w[J / 2] * shl[2]) & 0xC0C0C0C0u;  // i = 0: << 6
+    a2 = (w[J / 2] * shl[1]) & 0xC0C0C0C0u;  // i = 1: << 4
   } else {
-    a0 = (w[J / 2] >> (4 * (J % 2))) & 0x03030303u;
-    a2 = (w[J / 2] >> (4 * (J % 2) + 2)) & 0x03030303u;
+    a0 = (w[J / 2] * shl[0]) & 0xC0C0C0C0u;  // i = 2: << 2
+    a2 = w[J / 2] & 0xC0C0C0C0u;             // i = 3
   }
 }
+// log2 of the code multiple that i8_regs leaves at each width
+template <int R> constexpr int kI8CodeShift = R == 8 ? 0 : R == 4 ? 4 : 6;
 
 // One staged unit at width R on the integer path (one batch row, Tiling<1>):
 // the planes are loaded as for the bf16 path (128-byte swizzle); per chunk
@@ -647,9 +660,9 @@ __device__ __forceinline__ void i8_regs(const uint32_t (&w)[4], uint32_t& a0, ui
 // 16-byte load at xaddr + (s * J / 2 + jj) * xstep. MMA j accumulates into
 // chain j % 2.
 template <int R, int... Js>
-__device__ __forceinline__ void i8_chunk(const uint32_t (&lo)[2][2][4], const uint8_t* smem_base,
-                                         uint32_t xaddr, uint32_t xstep, int s, uint32_t* errp,
-                                         int (&ch)[2][2][4], std::integer_sequence<int, Js...>) {
+__device__ __forceinline__ void i8_chunk(const uint32_t (&lo)[2][2][4], const uint32_t (&shl)[3],
+                                         const uint8_t* smem_base, uint32_t xaddr, uint32_t xstep, int s,
+                                         uint32_t* errp, int (&ch)[2][2][4], std::integer_sequence<int, Js...>) {
   // the chunk's digit loads first, then its MMAs
   uint4 xbs[16 / R / 2];
 #pragma unroll
@@ -664,8 +677,8 @@ __device__ __forceinline__ void i8_chunk(const uint32_t (&lo)[2][2][4], const ui
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
       uint32_t a0, a1, a2, a3;
-      i8_regs<R, J>(lo[T][0], a0, a2);
-      i8_regs<R, J>(lo[T][1], a1, a3);
+      i8_regs<R, J>(lo[T][0], shl, a0, a2);
+      i8_regs<R, J>(lo[T][1], shl, a1, a3);
       mma_u8s8_16832(ch[T][J % 2], a0, a1, a2, a3, (J % 2) ? xb.z : xb.x, (J % 2) ? xb.w : xb.y);
     }
   };
@@ -674,7 +687,8 @@ __device__ __forceinline__ void i8_chunk(const uint32_t (&lo)[2][2][4], const ui
 
 template <int R>
 __device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xaddr, uint32_t xstep,
-                                                int warp, int lane, uint32_t* errp, int (&ch)[2][2][4]) {
+                                                int warp, int lane, const uint32_t (&shl)[3], uint32_t* errp,
+                                                int (&ch)[2][2][4]) {
   using TL = Tiling<1>;
   constexpr int TW = TL::TW, NSUB = TL::NSUB, P0 = TL::P0;
   const int g = lane >> 2, t = lane & 3;
@@ -696,7 +710,7 @@ __device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xad
   extern __shared__ __align__(128) uint8_t smem[];
 #pragma unroll
   for (int s = 0; s < NSUB; ++s)
-    i8_chunk<R>(lo[s], smem, xaddr, xstep, s, errp, ch, std::make_integer_sequence<int, 16 / R>{});
+    i8_chunk<R>(lo[s], shl, smem, xaddr, xstep, s, errp, ch, std::make_integer_sequence<int, 16 / R>{});
 }
 
 // run_segment for the integer kinds (one batch row). Each unit's header says
@@ -735,10 +749,11 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
           for (int j = 0; j < 4; ++j) { ch[T][0][j] = 0; ch[T][1][j] = 0; }
         const bool live = g < kI8Digits;
         process_unit_i8<R>(st, live ? xs + static_cast<uint32_t>(g * 4 + t) * 16u : zero_addr,
-                           live ? 4u * kI8Digits * 16u : 0u, warp, lane, p.err, ch);
-        // digit 2t weighs 2^(14t + E - 48), digit 2t + 1 2^(14t + 7 + E - 48)
-        const float w0 = __int_as_float((127 + 14 * t + E - 48) << 23);
-        const float w1 = __int_as_float((127 + 14 * t + 7 + E - 48) << 23);
+                           live ? 4u * kI8Digits * 16u : 0u, warp, lane, p.shl, p.err, ch);
+        // digit 2t weighs 2^(14t + E - 48), digit 2t + 1 2^(14t + 7 + E - 48);
+        // the codes came 2^kI8CodeShift times their value
+        const float w0 = __int_as_float((127 + 14 * t + E - 48 - kI8CodeShift<R>) << 23);
+        const float w1 = __int_as_float((127 + 14 * t + 7 + E - 48 - kI8CodeShift<R>) << 23);
 #pragma unroll
         for (int T = 0; T < 2; ++T) {
           tot[T][0][0] = fmaf(static_cast<float>(ch[T][0][0] + ch[T][1][0]), w0,
@@ -1111,7 +1126,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
   // biased exponent e, -133 for a subnormal) becomes X = m 2^(f + 48 - E),
   // below 2^49, an integer when f >= E - 48; digit g is (X >> 7g) & 127 with
   // x's sign. A unit with f < E - 48 somewhere, a non-finite input or E
-  // outside [-78, 100] gets the width's bf16 fragments and input sum instead
+  // outside [-72, 100] gets the width's bf16 fragments and input sum instead
   // (written by the digit-0 warp).
   if (p.n_i8 > 0) {
     const int lane = threadIdx.x & 31;
@@ -1167,7 +1182,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
         fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
       }
       const int E = emax == kNone ? 0 : emax;
-      if (emax != kNone && (fmin < E - 48 || E > 100 || E < -78)) bad = true;
+      if (emax != kNone && (fmin < E - 48 || E > 100 || E < -72)) bad = true;
       const bool fallback = __any_sync(0xffffffffu, bad);
       uint8_t* blk = L.xf + int64_t(kc) * i8_unit_bytes(r);
       const int64_t blk_end = int64_t(L.n_kc) * i8_unit_bytes(r);  // bytes of the layout
@@ -1414,11 +1429,11 @@ int64_t unit_cost(int dk) {
     case 6: return 183;
     case 10: case 11: return 110;  // one 8-bit plane, one MMA per 16 codes, more decode work
     // the integer kinds, from per-unit times of single-width stacks at one
-    // batch row on B200 (r = 8 streams near the HBM peak; r = 4 1.15x,
-    // r = 2 1.51x its unit time)
+    // batch row on B200 (r = 8 streams near the HBM peak; r = 4 1.09x,
+    // r = 2 1.24x its unit time)
     case kDkI8 + 8: return 100;
-    case kDkI8 + 4: return 115;
-    case kDkI8 + 2: return 151;
+    case kDkI8 + 4: return 109;
+    case kDkI8 + 2: return 124;
     default: return 301;  // 3
   }
 }
@@ -1647,6 +1662,9 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.pitch1 = P1;
   gp.err = err;
   gp.wait_ns = wait_limit_ns();
+  gp.shl[0] = 4u;
+  gp.shl[1] = 16u;
+  gp.shl[2] = 64u;
 
   switch (NT) {
     case 1: return i8_only ? launch_gemv<1, CAP, true>(gp, smem, grid, stream) : launch_gemv<1, CAP>(gp, smem, grid, stream);

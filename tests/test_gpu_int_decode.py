@@ -3,7 +3,7 @@ integer tensor cores: the codes are u8, and the prep kernel writes each input
 of a unit as the exact integer x 2^(48 - E) (E the unit's largest exponent) in
 seven signed 7-bit digits, one per MMA column. Inputs more than 41 octaves
 below the unit's largest, non-finite inputs, or a unit whose largest exponent
-lies outside [-78, 100] send that unit down the bf16 path instead. Either way
+lies outside [-72, 100] send that unit down the bf16 path instead. Either way
 y = x . W_r^T must hold within |y - y_ref| <= 1e-3 sum|x||W_r| + 1e-6 against
 the float64 oracle, whatever the spread of the inputs."""
 import numpy as np
@@ -77,10 +77,10 @@ def test_zeros_subnormals_and_single_nonzero(r):
 
 
 @pytest.mark.parametrize("r", WIDTHS)
-@pytest.mark.parametrize("e", [-90, -76, 90, 105])
+@pytest.mark.parametrize("e", [-90, -74, -70, 90, 105])
 def test_extreme_scales(r, e):
     """Units whose largest input is near the ends of the bf16 range: inside
-    [2^-78, 2^100] the digit weights stay normal fp32; outside, the unit falls
+    [2^-72, 2^100] the digit weights stay normal fp32; outside, the unit falls
     back to the bf16 path."""
     rng = np.random.default_rng(7)
     x = rng.standard_normal((1, 1024)) * 2.0 ** e
