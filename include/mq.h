@@ -70,7 +70,10 @@ MQ_API const char* mq_last_error(void);
 
 /*
  * Bytes of the dense r-bit planes of an N x K matrix: N*K*r/8.
- * Returns 0 for N < 1, K < 1, K % 32 != 0 or r not in {8, 6, 4, 3, 2}.
+ * Returns 0 for N < 1, r not in {8, 6, 4, 3, 2}, or K not a positive multiple
+ * of the width's K unit: every plane row (K*b/8 bytes for a plane of width b)
+ * must be a whole number of 16-byte units, so K % 32 at r = 8 and 4, K % 64
+ * at r = 6 and 2 (a 2-bit plane), K % 128 at r = 3 (a 1-bit plane).
  * Layout (this library's own; the pages fix only that a slice is an r-bit
  * integer per weight): r = 8 -> one plane of bytes (the container itself);
  * r = 4, 2 -> one plane of width r; r = 3 -> planes of widths (2, 1);
@@ -126,7 +129,8 @@ MQ_API mq_status mq_quantize_int8_clipped(const void* w, int dtype, int64_t N, i
  * decides the rounding, as the slicing paragraph states.
  *   q      : N x K uint8 container (from mq_quantize_int8), 16-byte aligned.
  *   packed : mq_packed_bytes(N, K, r) bytes out, 16-byte aligned.
- * Requires K % 32 == 0 and r in {8, 6, 4, 3, 2}.
+ * Requires r in {8, 6, 4, 3, 2} and K a multiple of the width's K unit (see
+ * mq_packed_bytes: 32, 64 or 128).
  */
 MQ_API mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r,
                         void* packed, void* stream);
@@ -140,9 +144,11 @@ MQ_API mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r,
  *   packed : planes of width r from mq_slice_pack, 16-byte aligned.
  *   alpha, zero : N fp32 (from mq_quantize_int8).
  *   y      : M x N fp32 out (overwritten), 4-byte aligned.
- * Requires 1 <= M, K % 128 == 0 (a 1-bit plane row must be a whole number of
- * 16-byte units for the bulk copies), N >= 1. M <= 32 runs the decode GEMV
- * (tensor-core m16n8k16 tiles fed from TMA-staged planes); M > 32 runs the
+ * Requires 1 <= M, N >= 1, and K a multiple of the width's K unit (32 at
+ * r = 8, 4; 64 at r = 6, 2; 128 at r = 3: every plane row a whole number of
+ * 16-byte units for the TMA boxes). M <= 32 runs the decode GEMV (legacy
+ * tensor-core tiles fed from TMA-staged planes: at M = 1 and r = 8, 4, 2 the
+ * integer m16n8k32 with exact sums, otherwise bf16 m16n8k16); M > 32 runs the
  * prefill GEMM (tcgen05, accumulators in tensor memory).
  * Accuracy: |y - y_exact| <= 1e-3 * sum_k |x[m,k]| |W_r[n,k]| + 1e-6.
  */
@@ -163,7 +169,7 @@ MQ_API mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* pack
  *   q : N x K uint8 container (row pitch K bytes), 16-byte aligned.
  *   Other arguments and the accuracy bound as mq_linear: M <= 32 runs the
  *   decode GEMV, larger M the prefill GEMM, both slicing while they decode.
- *   Requires K % 128 == 0, clamp in {0, 1}. At r = 8 both forms are the
+ *   Requires K % 32 == 0, clamp in {0, 1}. At r = 8 both forms are the
  *   container.
  */
 MQ_API mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t* q,
@@ -226,6 +232,14 @@ typedef struct mq_linear_desc {
  *   widths[n_layers]                  : HOST array, each in {8, 6, 4, 3, 2}.
  * Requires 1 <= M <= 32 and the mq_linear conditions for every linear.
  * Stacks longer than 256 linears are split into several launches.
+ * A launch of more than 8 linears reads their plane tensor maps from a device
+ * table: one per distinct list (device, planes addresses, N, K, widths),
+ * encoded and uploaded with an asynchronous copy on `stream` the first time
+ * the list is served, then reused. At most 64 tables (16 MiB) are kept; a new
+ * one evicts the least recently used, synchronizing that table's device
+ * before freeing it. A table served during a CUDA graph capture is pinned
+ * until mq_release_workspace (the graph holds its address); a list first seen
+ * during a capture returns MQ_ERR_CUDA (make one call before capturing).
  */
 MQ_API mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin,
                            int n_lins, const int* widths, int n_layers,
@@ -365,9 +379,19 @@ MQ_API mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, const vo
  */
 MQ_API mq_status mq_device_status(void* stream);
 
-/* Frees every workspace of this library (all devices and streams). The
- * caller must ensure no mq_* work is still in flight. */
+/* Frees every workspace of this library (all devices and streams) and its
+ * tensor-map tables (see mq_stack_forward). The caller must ensure no mq_*
+ * work is still in flight, and must not replay a CUDA graph that captured an
+ * mq_* call afterwards. */
 MQ_API mq_status mq_release_workspace(void);
+
+/*
+ * Testing hook: the number of tensor-map tables the library holds (a stack
+ * with more linears than fit in one launch's parameters reads its plane maps
+ * from a device table, one per distinct list of linears; at most 64 are kept,
+ * least recently used first out). Allocates nothing.
+ */
+MQ_API int64_t mq_debug_map_table_count(void);
 
 /*
  * Testing hook: the time (ns) a kernel waits on a pipeline barrier before it

@@ -91,6 +91,7 @@ _linear_noalloc = _sig("mq_linear_noalloc", _int,
 _device_status = _sig("mq_device_status", _int, [_vp])
 _release = _sig("mq_release_workspace", _int, [])
 _wait_limit = _sig("mq_debug_set_wait_limit_ns", _int, [_u64])
+_map_count = _sig("mq_debug_map_table_count", _i64, [])
 
 EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8",
             "mq_slice_pack", "mq_linear", "mq_stack_forward", "mq_device_status",
@@ -98,7 +99,7 @@ EXPORTED = ("mq_version", "mq_last_error", "mq_packed_bytes", "mq_quantize_int8"
             "mq_quantize_int8_clipped", "mq_linear_container", "mq_ep_overflow_rows",
             "mq_ep_overflow_cols", "mq_linear_ep", "mq_chain_scratch_bytes",
             "mq_chain_forward", "mq_container_save", "mq_container_info", "mq_container_load",
-            "mq_chain_scratch_views")
+            "mq_chain_scratch_views", "mq_debug_map_table_count")
 
 NOALLOC_SCRATCH_BYTES = 1280 * 1024
 
@@ -301,6 +302,10 @@ def release_workspace() -> None:
 
 def debug_set_wait_limit_ns(ns: int) -> None:
     _check(_wait_limit(ns))
+
+
+def debug_map_table_count() -> int:
+    return int(_map_count())
 
 
 def raw_status(fn_name: str, *args) -> int:

@@ -54,6 +54,13 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool valid_r(int r) { return r == 8 || r == 6 || r == 4 || r == 3 || r == 2; }
 
+// The K a width's planes need: every plane row (K b / 8 bytes for a plane of
+// width b) must be a whole number of 16-byte units, the row pitch of a TMA
+// box. r = 8 and 4 need K % 32 (with the pages' K % 32 as the floor), r = 6
+// and 2 (a 2-bit plane) K % 64, r = 3 (a 1-bit plane) K % 128. The int8
+// container (one byte per weight) serves every width from K % 32.
+int plane_kmult(int r) { return r == 3 ? 128 : (r == 6 || r == 2) ? 64 : 32; }
+
 }  // namespace
 
 int sm_count() {
@@ -133,7 +140,7 @@ int mq_version(void) { return (0 << 16) | 3; }
 const char* mq_last_error(void) { return g_last_error.c_str(); }
 
 size_t mq_packed_bytes(int64_t N, int64_t K, int r) {
-  if (N < 1 || K < 1 || K % 32 != 0 || !valid_r(r)) return 0;
+  if (N < 1 || K < 1 || !valid_r(r) || K % plane_kmult(r) != 0) return 0;
   return static_cast<size_t>(N) * static_cast<size_t>(K) * static_cast<size_t>(r) / 8;
 }
 
@@ -176,7 +183,9 @@ mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* pac
   g_last_error.clear();
   if (!q || !packed) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: null pointer");
   if (!valid_r(r)) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: r=%d not in {8,6,4,3,2}", r);
-  if (N < 1 || K < 1 || K % 32 != 0) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: need N >= 1 and K a positive multiple of 32 (K=%lld)", (long long)K);
+  if (N < 1 || K < 1 || K % plane_kmult(r) != 0)
+    return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: need N >= 1 and K a positive multiple of %d at r = %d (K=%lld)",
+                plane_kmult(r), r, (long long)K);
   if (!aligned(q, 16) || !aligned(packed, 16)) return fail(MQ_ERR_INVALID_ARG, "mq_slice_pack: q and packed must be 16-byte aligned");
   if (N * K > (int64_t(1) << 40)) return fail(MQ_ERR_UNSUPPORTED, "mq_slice_pack: matrix too large");
   cudaError_t e = launch_slice_pack(q, N, K, r, packed, static_cast<cudaStream_t>(stream), sm_count());
@@ -184,13 +193,18 @@ mq_status mq_slice_pack(const uint8_t* q, int64_t N, int64_t K, int r, void* pac
   return MQ_OK;
 }
 
+// kmult: the K multiple the weights' layout needs (plane_kmult(r) for
+// planes, 32 for the container).
 static mq_status check_linear(const char* who, const void* x, int64_t M, int64_t K, const void* packed,
-                              const float* alpha, const float* zero, int64_t N, int r, const float* y) {
+                              const float* alpha, const float* zero, int64_t N, int r, const float* y,
+                              int kmult) {
   if (!x || !packed || !alpha || !zero || !y) return fail(MQ_ERR_INVALID_ARG, "%s: null pointer", who);
   if (!valid_r(r)) return fail(MQ_ERR_INVALID_ARG, "%s: r=%d not in {8,6,4,3,2}", who, r);
   if (M < 1) return fail(MQ_ERR_INVALID_ARG, "%s: M must be >= 1", who);
   if (N < 1) return fail(MQ_ERR_INVALID_ARG, "%s: N must be >= 1", who);
-  if (K < 128 || K % 128 != 0) return fail(MQ_ERR_INVALID_ARG, "%s: K must be a positive multiple of 128 (K=%lld)", who, (long long)K);
+  if (K < kmult || K % kmult != 0)
+    return fail(MQ_ERR_INVALID_ARG, "%s: K must be a positive multiple of %d at r = %d (K=%lld)", who, kmult, r,
+                (long long)K);
   if (!aligned(x, 16) || !aligned(packed, 16)) return fail(MQ_ERR_INVALID_ARG, "%s: x and packed must be 16-byte aligned", who);
   if (!aligned(alpha, 4) || !aligned(zero, 4) || !aligned(y, 4)) return fail(MQ_ERR_INVALID_ARG, "%s: alpha, zero, y must be 4-byte aligned", who);
   if (N > (int64_t(1) << 30) || K > (int64_t(1) << 24)) return fail(MQ_ERR_UNSUPPORTED, "%s: N or K too large", who);
@@ -201,7 +215,7 @@ mq_status mq_linear(const void* x, int64_t M, int64_t K, const void* packed, con
                     const float* zero, int64_t N, int r, float* y, void* stream) {
   TraceRange trace_("mq_linear");
   g_last_error.clear();
-  mq_status st = check_linear("mq_linear", x, M, K, packed, alpha, zero, N, r, y);
+  mq_status st = check_linear("mq_linear", x, M, K, packed, alpha, zero, N, r, y, valid_r(r) ? plane_kmult(r) : 32);
   if (st != MQ_OK) return st;
   LinearJob job{x, static_cast<const uint8_t*>(packed), alpha, zero, y, N, K, r};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -222,7 +236,7 @@ mq_status mq_linear_container(const void* x, int64_t M, int64_t K, const uint8_t
                               float* y, void* stream) {
   TraceRange trace_("mq_linear_container");
   g_last_error.clear();
-  mq_status st = check_linear("mq_linear_container", x, M, K, q, alpha, zero, N, r, y);
+  mq_status st = check_linear("mq_linear_container", x, M, K, q, alpha, zero, N, r, y, 32);
   if (st != MQ_OK) return st;
   if (clamp != 0 && clamp != 1) return fail(MQ_ERR_INVALID_ARG, "mq_linear_container: clamp must be 0 or 1");
   LinearJob job{x, q, alpha, zero, y, N, K, r, clamp ? kContainer : kContainerEP};
@@ -278,7 +292,7 @@ mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed, 
                        const uint16_t* cols, float* y, void* stream) {
   TraceRange trace_("mq_linear_ep");
   g_last_error.clear();
-  mq_status st = check_linear("mq_linear_ep", x, M, K, packed, alpha, zero, N, r, y);
+  mq_status st = check_linear("mq_linear_ep", x, M, K, packed, alpha, zero, N, r, y, valid_r(r) ? plane_kmult(r) : 32);
   if (st != MQ_OK) return st;
   if (r == 8) return fail(MQ_ERR_INVALID_ARG, "mq_linear_ep: r=8 has no extra bucket");
   if (!row_ptr || !cols || !aligned(row_ptr, 4) || !aligned(cols, 2))
@@ -331,7 +345,8 @@ mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, int64_t M
       char w[64];
       std::snprintf(w, sizeof(w), "%s[layer %d, linear %d]", who, l, i);
       // a 16-byte-aligned stand-in for x: the chain's own bf16 buffers
-      mq_status st = check_linear(w, scratch, M, nin[i], L.packed[i], L.alpha[i], L.zero[i], nout[i], L.r, h);
+      mq_status st = check_linear(w, scratch, M, nin[i], L.packed[i], L.alpha[i], L.zero[i], nout[i], L.r, h,
+                                  valid_r(L.r) ? plane_kmult(L.r) : 32);
       if (st != MQ_OK) return st;
     }
   }
@@ -388,7 +403,7 @@ mq_status mq_stack_forward(const mq_linear_desc* lins, const int* layer_of_lin, 
     const mq_linear_desc& d = lins[i];
     char who[64];
     std::snprintf(who, sizeof(who), "mq_stack_forward[lin %d]", i);
-    mq_status st = check_linear(who, d.x, M, d.K, d.packed, d.alpha, d.zero, d.N, r, d.y);
+    mq_status st = check_linear(who, d.x, M, d.K, d.packed, d.alpha, d.zero, d.N, r, d.y, valid_r(r) ? plane_kmult(r) : 32);
     if (st != MQ_OK) return st;
     jobs[i] = LinearJob{d.x, static_cast<const uint8_t*>(d.packed), d.alpha, d.zero, d.y, d.N, d.K, r};
   }
@@ -446,8 +461,11 @@ mq_status mq_release_workspace(void) {
   g_workspaces.clear();
   cudaSetDevice(cur);
   release_chain_graphs();
+  release_map_tables();
   return MQ_OK;
 }
+
+int64_t mq_debug_map_table_count(void) { return static_cast<int64_t>(map_table_count()); }
 
 mq_status mq_debug_set_wait_limit_ns(uint64_t ns) {
   g_last_error.clear();

@@ -206,7 +206,9 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
-  const int n_k = p.K / kBK;
+  // a ragged last stage reads past K: the TMA boxes fill it with zeros, and a
+  // zero input times any decoded weight adds nothing
+  const int n_k = (p.K + kBK - 1) / kBK;
   constexpr int kDecodeWarps = 8;   // per stage: one of the two decode groups
 
   if (threadIdx.x == 0) {
@@ -438,7 +440,7 @@ cudaError_t launch_gemm_r(const GemmParams& gp, dim3 grid, size_t smem, cudaStre
 }  // namespace
 
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
-  if (M < 1 || job.K % kBK != 0 || job.N < 1) return cudaErrorNotSupported;
+  if (M < 1 || job.K < 32 || job.K % 32 != 0 || job.N < 1) return cudaErrorNotSupported;
   if ((job.N + kBN - 1) / kBN > 0x7FFFFFFF || (M + kBM - 1) / kBM > 65535) return cudaErrorNotSupported;
   int b0, b1;
   job_planes(job, b0, b1);

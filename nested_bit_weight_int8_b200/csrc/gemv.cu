@@ -64,6 +64,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <list>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -178,14 +179,6 @@ template <> struct Geo<6> { static constexpr int b0 = 4, b1 = 2, W8 = 4; };
 // 8-bit plane.
 template <> struct Geo<10> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
 template <> struct Geo<11> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
-
-// bf16x2 of a small positive integer v (at most 8 significant bits, exact)
-// in both halves.
-__host__ __device__ constexpr uint32_t bf16x2_int(int v) {
-  int e = 0;
-  while ((2 << e) <= v) ++e;
-  return ((static_cast<uint32_t>(127 + e) << 7) | ((static_cast<uint32_t>(v) << (7 - e)) & 0x7Fu)) * 0x10001u;
-}
 
 // Per-linear constants of the slice-on-load decode (both 16-bit halves):
 // h2 the rounding addend 2^(s-1), kmask the code's bits after the shift, mag
@@ -1148,7 +1141,8 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       // (a) E, the smallest exponent f and non-finite inputs over the unit
       int emax = kNone, fmin = 1 << 30;
       bool bad = false;
-      const int ept = KC / 32;  // 4, 8 or 16 consecutive inputs per lane (K % 128 == 0: all in or all out)
+      const int ept = KC / 32;  // 4, 8 or 16 consecutive inputs per lane (all in or all out: K % 32
+                                // at r = 8 and 4, K % 64 at r = 2)
       const int64_t k0 = kbase + int64_t(lane) * ept;
       uint32_t xe[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
       if (k0 < L.K) {  // all loads first
@@ -1195,7 +1189,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
           const int s = lane / (4 * J2), jj = (lane / 4) % J2, t = lane % 4;
           const int64_t k16 = kbase + int64_t(4 * s + t) * cpc + 16 * jj;
           uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          if (k16 < L.K) {  // the chunk lies wholly inside or outside K (K % 128 == 0)
+          if (k16 < L.K) {  // the 16 inputs lie wholly inside or outside K (K % 32 == 0)
             const uint4 va = *reinterpret_cast<const uint4*>(xr + k16);
             const uint4 vb = *reinterpret_cast<const uint4*>(xr + k16 + 8);
             xw[0] = va.x; xw[1] = va.y; xw[2] = va.z; xw[3] = va.w;
@@ -1362,12 +1356,6 @@ cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int grid, cudaSt
   return cudaLaunchKernelEx(&cfg, kern, gp);
 }
 
-// Device tables of tensor maps for large launches, one per distinct list of
-// (planes address, N, K, r) and box width. Built with a synchronous copy the
-// first time a stack is served (so the first call must not be captured),
-// then reused by every later identical call.
-std::map<std::pair<int, std::vector<uint64_t>>, CUtensorMap*> g_map_tables;
-
 cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
   int b0, b1;
   job_planes(j, b0, b1);
@@ -1380,9 +1368,53 @@ cudaError_t encode_plane_maps(const LinearJob& j, int P0, CUtensorMap* out2) {
                        uint64_t(j.K) * b1 / 8, static_cast<uint32_t>(P0 / 2), rows, 1);
 }
 
-cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUtensorMap** out) {
+// Device tables of tensor maps for launches with more linears than fit in
+// the kernel parameters: one table per distinct (device, box width, list of
+// planes address, N, K, r), uploaded on the call's stream the first time that
+// list is served and reused by every later identical call.
+//
+// The cache is bounded: at most kMaxMapTables tables and kMaxMapBytes bytes.
+// A new table evicts the least recently used ones; since an evicted table may
+// still be read by a launch in flight, eviction synchronizes that table's
+// device before freeing it. A table served to a call that is being captured
+// into a CUDA graph is pinned (the graph holds its address) and stays until
+// mq_release_workspace. A list first seen during a capture is refused: its
+// upload would have to become part of the graph.
+constexpr size_t kMaxMapTables = 64;
+constexpr size_t kMaxMapBytes = size_t(16) << 20;
+
+using MapKey = std::pair<int, std::vector<uint64_t>>;
+struct MapTable {
+  CUtensorMap* dptr;
+  size_t bytes;
+  bool pinned;
+  std::list<const MapKey*>::iterator lru;  // position in g_map_lru (front: most recent)
+};
+std::map<MapKey, MapTable> g_map_tables;
+std::list<const MapKey*> g_map_lru;
+size_t g_map_bytes = 0;
+
+// Frees one table after its device has finished all work. Caller holds
+// g_cache_mutex.
+void free_map_table(std::map<MapKey, MapTable>::iterator it) {
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != it->first.first) cudaSetDevice(it->first.first);
+  cudaDeviceSynchronize();
+  cudaFree(it->second.dptr);
+  if (cur != it->first.first) cudaSetDevice(cur);
+  g_map_bytes -= it->second.bytes;
+  g_map_lru.erase(it->second.lru);
+  g_map_tables.erase(it);
+}
+
+cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, cudaStream_t stream,
+                          const CUtensorMap** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cap);
   if (e != cudaSuccess) return e;
   std::vector<uint64_t> key;
   key.reserve(size_t(n_jobs) * 4 + 1);
@@ -1394,27 +1426,65 @@ cudaError_t get_map_table(const LinearJob* jobs, int n_jobs, int P0, const CUten
     key.push_back(uint64_t(jobs[i].r) | (uint64_t(jobs[i].src) << 8));
   }
   std::lock_guard<std::mutex> lk(g_cache_mutex);
-  auto k2 = std::make_pair(dev, std::move(key));
+  MapKey k2(dev, std::move(key));
   auto it = g_map_tables.find(k2);
   if (it != g_map_tables.end()) {
-    *out = it->second;
+    g_map_lru.splice(g_map_lru.begin(), g_map_lru, it->second.lru);
+    if (cap != cudaStreamCaptureStatusNone) it->second.pinned = true;
+    *out = it->second.dptr;
     return cudaSuccess;
   }
+  if (cap != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
+
+  const size_t bytes = size_t(n_jobs) * 2 * sizeof(CUtensorMap);
   std::vector<CUtensorMap> host(size_t(n_jobs) * 2);
-  std::memset(host.data(), 0, host.size() * sizeof(CUtensorMap));
+  std::memset(host.data(), 0, bytes);
   for (int i = 0; i < n_jobs; ++i) {
     e = encode_plane_maps(jobs[i], P0, &host[size_t(2) * i]);
     if (e != cudaSuccess) return e;
   }
+  // evict from the least recent end, passing over pinned tables
+  auto victim = g_map_lru.end();
+  while ((g_map_tables.size() >= kMaxMapTables || g_map_bytes + bytes > kMaxMapBytes) &&
+         victim != g_map_lru.begin()) {
+    --victim;
+    auto vt = g_map_tables.find(**victim);
+    if (vt->second.pinned) continue;
+    auto next = std::next(victim);
+    free_map_table(vt);
+    victim = next;
+  }
   CUtensorMap* dptr = nullptr;
-  e = cudaMalloc(&dptr, host.size() * sizeof(CUtensorMap));
+  e = cudaMalloc(&dptr, bytes);
   if (e != cudaSuccess) return e;
-  e = cudaMemcpy(dptr, host.data(), host.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) { cudaFree(dptr); return e; }
-  g_map_tables.emplace(std::move(k2), dptr);
+  // from pageable memory: the call returns once `host` has been staged
+  e = cudaMemcpyAsync(dptr, host.data(), bytes, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) {
+    cudaFree(dptr);
+    return e;
+  }
+  auto ins = g_map_tables.emplace(std::move(k2), MapTable{dptr, bytes, false, {}}).first;
+  g_map_lru.push_front(&ins->first);
+  ins->second.lru = g_map_lru.begin();
+  g_map_bytes += bytes;
   *out = dptr;
   return cudaSuccess;
 }
+
+}  // namespace
+
+// Frees every tensor-map table (all devices), after their devices finish.
+void release_map_tables() {
+  std::lock_guard<std::mutex> lk(g_cache_mutex);
+  while (!g_map_tables.empty()) free_map_table(g_map_tables.begin());
+}
+
+size_t map_table_count() {
+  std::lock_guard<std::mutex> lk(g_cache_mutex);
+  return g_map_tables.size();
+}
+
+namespace {
 
 // Relative cost of one unit of each width, for cutting the CTA ranges. A unit
 // always holds the same plane bytes per row (two planes hold 1.5x), while the
@@ -1511,7 +1581,7 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     }
     gp.map_table = nullptr;
   } else {
-    cudaError_t em = get_map_table(jobs, n_jobs, P0, &gp.map_table);
+    cudaError_t em = get_map_table(jobs, n_jobs, P0, stream, &gp.map_table);
     if (em != cudaSuccess) return em;
   }
   const size_t psum_off = xf_bytes;

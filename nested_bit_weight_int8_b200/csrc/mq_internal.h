@@ -155,6 +155,10 @@ void chain_views(int64_t M, int64_t D, int64_t Dkv, int64_t F, size_t out[10]);
 cudaError_t run_chain(const struct mq_chain_layer* layers, int n_layers, int M, int D, int Dkv, int F,
                       int hd, float* h, void* scratch, bool use_graph, cudaStream_t stream);
 void release_chain_graphs();
+// The bounded cache of tensor-map tables of large decode launches: frees all
+// of it (after the devices finish), and its current size.
+void release_map_tables();
+size_t map_table_count();
 
 // Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
 // cudaErrorNotSupported for shapes it does not serve (nothing launched).

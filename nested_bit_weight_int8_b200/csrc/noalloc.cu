@@ -96,8 +96,11 @@ extern "C" mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, cons
     return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: r=%d not in {8,6,4,3,2}", r);
   if (M < 1 || M > 32) return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: M=%lld must be in [1, 32]", (long long)M);
   if (N < 1) return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: N must be >= 1");
-  if (K < 128 || K % 128 != 0)
-    return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: K must be a positive multiple of 128 (K=%lld)", (long long)K);
+  // every plane row a whole number of 16-byte units (as mq_linear)
+  const int kmult = r == 3 ? 128 : (r == 6 || r == 2) ? 64 : 32;
+  if (K < kmult || K % kmult != 0)
+    return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: K must be a positive multiple of %d at r = %d (K=%lld)",
+                        kmult, r, (long long)K);
   if (!aligned(x, 16) || !aligned(packed, 16))
     return noalloc_fail(MQ_ERR_INVALID_ARG, "mq_linear_noalloc: x and packed must be 16-byte aligned");
   if (!aligned(alpha, 4) || !aligned(zero, 4) || !aligned(y, 4))

@@ -39,7 +39,30 @@ def test_version():
 @pytest.mark.parametrize("r", [8, 6, 4, 3, 2])
 def test_packed_bytes(r):
     assert mq.packed_bytes(14336, 4096, r) == 14336 * 4096 * r // 8
-    assert mq.packed_bytes(1, 32, r) == 4 * r
+    assert mq.packed_bytes(1, 32, r) == (4 * r if r in (8, 4) else 0)
+    assert mq.packed_bytes(1, 128, r) == 16 * r
+
+
+# the K unit of each width: every plane row a whole number of 16-byte units
+K_UNIT = {8: 32, 4: 32, 6: 64, 2: 64, 3: 128}
+
+
+@pytest.mark.parametrize("r", [8, 6, 4, 3, 2])
+def test_k_unit_per_width(r):
+    u = K_UNIT[r]
+    F = FAKE
+    for k in (u, 3 * u, 4096 + u):
+        assert mq.packed_bytes(4, k, r) == 4 * k * r // 8
+    for k in (u // 2, u + 16, 3 * u - 16, 4096 + u // 2):
+        if k % K_UNIT[r] == 0:
+            continue
+        assert mq.packed_bytes(4, k, r) == 0, (r, k)
+        assert mq.raw_status("mq_slice_pack", F, 4, k, r, F, None) == mq.MQ_ERR_INVALID_ARG, (r, k)
+        assert mq.raw_status("mq_linear", F, 1, k, F, F, F, 64, r, F, None) == mq.MQ_ERR_INVALID_ARG, (r, k)
+        assert f"multiple of {u}" in mq.last_error()
+    # the int8 container serves every width from K % 32
+    assert mq.raw_status("mq_linear_container", F, 1, 80, F, F, F, 64, r, 1, F, None) == mq.MQ_ERR_INVALID_ARG
+    assert "multiple of 32" in mq.last_error()
 
 
 def test_packed_bytes_rejects():
@@ -67,7 +90,9 @@ def test_linear_rejects_bad_shapes_and_pointers():
     F = FAKE
     cases = [
         (F, 0, 256, F, F, F, 64, 4, F),      # M = 0
-        (F, 1, 96, F, F, F, 64, 4, F),       # K % 128
+        (F, 1, 80, F, F, F, 64, 4, F),       # K % 32 at r = 4
+        (F, 1, 96, F, F, F, 64, 2, F),       # K % 64 at r = 2
+        (F, 1, 192, F, F, F, 64, 3, F),      # K % 128 at r = 3
         (F, 1, 0, F, F, F, 64, 4, F),        # K = 0
         (F, 1, 256, F, F, F, 0, 4, F),       # N = 0
         (None, 1, 256, F, F, F, 64, 4, F),   # null x
@@ -114,7 +139,7 @@ def test_linear_container_rejects():
     bad = [
         ((F, 1, 256, F, F, F, 64, 5, 1, F), mq.MQ_ERR_INVALID_ARG),    # r
         ((F, 1, 256, F, F, F, 64, 4, 2, F), mq.MQ_ERR_INVALID_ARG),    # clamp not 0/1
-        ((F, 1, 96, F, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),     # K % 128
+        ((F, 1, 80, F, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),     # K % 32
         ((F, 1, 256, F + 4, F, F, 64, 4, 1, F), mq.MQ_ERR_INVALID_ARG),  # misaligned q
         ((F, 1, 256, None, F, F, 64, 4, 0, F), mq.MQ_ERR_INVALID_ARG),   # null q
     ]

@@ -54,9 +54,10 @@ def test_noalloc_matches_linear_on_consecutive_calls():
     # fixed array serves, with another width and shape, so it reuses the
     # array after the first call left its own contents there. The last two
     # are r = 2 at one batch row (inputs staged as integer digits), the
-    # largest K of that layout last.
+    # largest K of that layout last; then K a multiple of 32 or 64 only.
     cases = [(8, 2048, 4096, 4, 31), (32, 1000, 16384, 2, 32), (1, 777, 2304, 8, 33),
-             (1, 1500, 8192, 2, 34), (1, 64, 183808, 2, 35)]
+             (1, 1500, 8192, 2, 34), (1, 64, 183808, 2, 35),
+             (1, 300, 96, 4, 36), (3, 200, 4160, 2, 37)]   # K on the width's own unit (32, 64)
     for M, N, K, r, seed in cases:
         w = synth.f32_from_bf16_bits(synth.gaussian_weights(N, K, seed)).astype(np.float64)
         q, a, z = oracle.quantize_minmax(w)
