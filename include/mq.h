@@ -318,6 +318,12 @@ MQ_API mq_status mq_chain_forward(const mq_chain_layer* layers, int n_layers, in
  * below 1, or a file of another shape (load); MQ_ERR_IO for a file that
  * cannot be opened, written or read, is truncated, has trailing bytes, is not
  * a container of this version, or fails its checksum.
+ * mq_container_save writes the file under a temporary name beside `path`
+ * (path.tmp.<pid>), checks that it closed cleanly, then renames it over
+ * `path`: readers see the old file or the complete new one, and a failed save
+ * leaves `path` untouched. mq_container_load reads straight into q, alpha and
+ * zero; if it returns an error, their contents are undefined (partly
+ * overwritten).
  */
 MQ_API mq_status mq_container_save(const char* path, const uint8_t* q, const float* alpha,
                                    const float* zero, int64_t N, int64_t K);

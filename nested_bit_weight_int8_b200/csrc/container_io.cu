@@ -16,6 +16,9 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <string>
+
+#include <unistd.h>
 
 #include "../../include/mq.h"
 #include "mq_internal.h"
@@ -68,11 +71,16 @@ struct File {
 
 }  // namespace
 
+// Writes the whole file under a temporary name beside `path` (path.tmp.<pid>),
+// closes it, and only then renames it over `path`: a reader sees the old file
+// or the complete new one, never a partial write, and a failed save leaves
+// `path` as it was.
 int container_save(const char* path, const uint8_t* q, const float* alpha, const float* zero, int64_t N,
                    int64_t K, char* why, size_t why_len) {
   if (!host_little_endian()) { std::snprintf(why, why_len, "big-endian hosts are not supported"); return 1; }
-  File fh(path, "wb");
-  if (!fh.f) { std::snprintf(why, why_len, "cannot open %s for writing", path); return 1; }
+  const std::string tmp = std::string(path) + ".tmp." + std::to_string(static_cast<long long>(getpid()));
+  std::FILE* f = std::fopen(tmp.c_str(), "wb");
+  if (!f) { std::snprintf(why, why_len, "cannot open %s for writing", tmp.c_str()); return 1; }
   const Crc32& T = crc_table();
   uint8_t header[kHeaderBytes];
   std::memcpy(header, kMagic, 4);
@@ -80,17 +88,27 @@ int container_save(const char* path, const uint8_t* q, const float* alpha, const
   std::memcpy(header + 8, &N, 8);
   std::memcpy(header + 16, &K, 8);
   uint32_t crc = T.update(0, header, sizeof(header));
-  bool ok = std::fwrite(header, 1, sizeof(header), fh.f) == sizeof(header);
+  bool ok = std::fwrite(header, 1, sizeof(header), f) == sizeof(header);
   const size_t nq = static_cast<size_t>(N) * static_cast<size_t>(K);
-  ok = ok && std::fwrite(q, 1, nq, fh.f) == nq;
+  ok = ok && std::fwrite(q, 1, nq, f) == nq;
   crc = T.update(crc, q, nq);
-  ok = ok && std::fwrite(alpha, 4, static_cast<size_t>(N), fh.f) == static_cast<size_t>(N);
+  ok = ok && std::fwrite(alpha, 4, static_cast<size_t>(N), f) == static_cast<size_t>(N);
   crc = T.update(crc, alpha, 4 * static_cast<size_t>(N));
-  ok = ok && std::fwrite(zero, 4, static_cast<size_t>(N), fh.f) == static_cast<size_t>(N);
+  ok = ok && std::fwrite(zero, 4, static_cast<size_t>(N), f) == static_cast<size_t>(N);
   crc = T.update(crc, zero, 4 * static_cast<size_t>(N));
-  ok = ok && std::fwrite(&crc, 4, 1, fh.f) == 1;
-  ok = ok && std::fflush(fh.f) == 0;
-  if (!ok) { std::snprintf(why, why_len, "write to %s failed", path); return 1; }
+  ok = ok && std::fwrite(&crc, 4, 1, f) == 1;
+  ok = ok && std::fflush(f) == 0;
+  ok = (std::fclose(f) == 0) && ok;  // fclose reports errors of buffered writes too
+  if (!ok) {
+    std::remove(tmp.c_str());
+    std::snprintf(why, why_len, "write to %s failed", tmp.c_str());
+    return 1;
+  }
+  if (std::rename(tmp.c_str(), path) != 0) {
+    std::remove(tmp.c_str());
+    std::snprintf(why, why_len, "cannot rename %s to %s", tmp.c_str(), path);
+    return 1;
+  }
   return 0;
 }
 

@@ -80,3 +80,31 @@ def test_shape_mismatch_and_bad_arguments(tmp_path):
     with pytest.raises(mq.MQError) as e:
         mq.container_shape(str(tmp_path / "missing.mqc"))
     assert e.value.status == mq.MQ_ERR_IO
+
+
+def test_save_replaces_atomically_and_leaves_no_temporary(tmp_path):
+    """A save writes path.tmp.<pid>, closes it and renames it over path: an
+    existing file is replaced whole, and no temporary stays behind."""
+    q, a, z = _container(11, 64, 4)
+    p = str(tmp_path / "c.mqc")
+    mq.save_container(p, q, a, z)
+    q2, a2, z2 = _container(11, 64, 5)
+    mq.save_container(p, q2, a2, z2)
+    assert sorted(os.listdir(tmp_path)) == ["c.mqc"]
+    q3, _, _ = mq.load_container(p)
+    assert torch.equal(q3, q2)
+
+
+def test_failed_save_leaves_the_target_untouched(tmp_path):
+    """When the rename cannot happen (the target is a non-empty directory),
+    the save fails with MQ_ERR_IO, the target is as it was and the temporary
+    file is removed."""
+    q, a, z = _container(7, 32, 6)
+    target = tmp_path / "c.mqc"
+    target.mkdir()
+    (target / "keep").write_bytes(b"x")
+    with pytest.raises(mq.MQError) as e:
+        mq.save_container(str(target), q, a, z)
+    assert e.value.status == mq.MQ_ERR_IO
+    assert sorted(os.listdir(tmp_path)) == ["c.mqc"]
+    assert (target / "keep").read_bytes() == b"x"
