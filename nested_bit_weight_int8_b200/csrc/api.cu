@@ -75,10 +75,11 @@ int sm_count() {
   return n;
 }
 
-cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out) {
+cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out, uint32_t** sync) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  bytes += kSyncBytes;
   std::lock_guard<std::mutex> lk(g_ws_mutex);
   Workspace& w = g_workspaces[std::make_pair(dev, stream)];
   if (w.bytes < bytes) {
@@ -94,8 +95,12 @@ cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out) {
     e = cudaMalloc(&w.ptr, sz);
     if (e != cudaSuccess) return e;
     w.bytes = sz;
+    // the barrier words start at zero, ahead of any kernel on this stream
+    e = cudaMemsetAsync(w.ptr, 0, kSyncBytes, stream);
+    if (e != cudaSuccess) return e;
   }
-  *out = w.ptr;
+  *out = static_cast<uint8_t*>(w.ptr) + kSyncBytes;
+  if (sync) *sync = static_cast<uint32_t*>(w.ptr);
   return cudaSuccess;
 }
 

@@ -34,15 +34,17 @@ constexpr int kGlueThreads = 256;
 constexpr float kEps = 1e-6f;
 
 // One CTA per batch row: v = h + add (add may be null), written to h_out if
-// given; xn = bf16(v / sqrt(mean(v^2) + eps)) if xn is given.
+// given; xn = bf16(v / sqrt(mean(v^2) + eps)) if xn is given. `clear` (may be
+// null) is a word set to zero once the previous grid has finished.
 __global__ void __launch_bounds__(kGlueThreads)
 rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ add, float* __restrict__ h_out,
-               __nv_bfloat16* __restrict__ xn, int D) {
+               __nv_bfloat16* __restrict__ xn, int D, uint32_t* clear) {
   __shared__ float red[kGlueThreads / 32];
   __shared__ float s_inv;
   pdl_launch_dependents();
   pdl_wait_primary();
   const int m = blockIdx.x, tid = threadIdx.x;
+  if (clear && m == 0 && tid == 0) *clear = 0u;
   const float* hr = h + int64_t(m) * D;
   const float* ar = add ? add + int64_t(m) * D : nullptr;
   float ss = 0.f;
@@ -108,7 +110,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 // Byte offsets of the chain's buffers inside the caller's scratch.
 struct ChainLayout {
-  size_t xn, qkv, a, o, h1, xn1, g, u, act, dn, ws, ws_bytes, total;
+  size_t xn, qkv, a, o, h1, xn1, g, u, act, dn, ws, ws_bytes, sync, total;
 };
 
 ChainLayout chain_layout(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
@@ -139,6 +141,9 @@ ChainLayout chain_layout(int64_t M, int64_t D, int64_t Dkv, int64_t F) {
   }
   L.ws_bytes = align256(need);
   L.ws = take(L.ws_bytes);
+  // grid-barrier words of the short integer decode launches (the arrival
+  // count is cleared by the chain's first kernel on every call)
+  L.sync = take(256);
   L.total = off;
   return L;
 }
@@ -156,7 +161,8 @@ struct ChainArgs {
 cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t s, int sms) {
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(c.scratch + off); };
   auto fp = [&](size_t off) { return reinterpret_cast<float*>(c.scratch + off); };
-  const FixedScratch fx{c.scratch + L.ws, L.ws_bytes, c.err};
+  uint32_t* sync = reinterpret_cast<uint32_t*>(c.scratch + L.sync);
+  const FixedScratch fx{c.scratch + L.ws, L.ws_bytes, c.err, sync};
   const int M = c.M, D = c.D, Dkv = c.Dkv, F = c.F;
   cudaError_t e;
   // xn = bf16(rmsnorm(h)) for the first layer; later layers get it from the
@@ -164,7 +170,7 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
   const float* no_add = nullptr;
   float* no_out = nullptr;
   e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(c.h), no_add,
-                 no_out, bf(L.xn), D);
+                 no_out, bf(L.xn), D, sync);
   if (e != cudaSuccess) return e;
   for (int l = 0; l < c.n_layers; ++l) {
     const mq_chain_layer& Ly = c.layers[l];
@@ -188,7 +194,7 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
     LinearJob jo = job(1, bf(L.a), D, D, fp(L.o));
     if ((e = run_gemv_fixed_n(&jo, 1, M, s, fx)) != cudaSuccess) return e;
     e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(c.h),
-                   static_cast<const float*>(fp(L.o)), fp(L.h1), bf(L.xn1), D);
+                   static_cast<const float*>(fp(L.o)), fp(L.h1), bf(L.xn1), D, static_cast<uint32_t*>(nullptr));
     if (e != cudaSuccess) return e;
     LinearJob jgu[2] = {job(2, bf(L.xn1), F, D, fp(L.g)), job(3, bf(L.xn1), F, D, fp(L.u))};
     if ((e = run_gemv_fixed_n(jgu, 2, M, s, fx)) != cudaSuccess) return e;
@@ -202,7 +208,7 @@ cudaError_t enqueue_chain(const ChainArgs& c, const ChainLayout& L, cudaStream_t
     // last layer, whose intermediates then all stay in the scratch)
     __nv_bfloat16* next_xn = l + 1 < c.n_layers ? bf(L.xn) : nullptr;
     e = launch_pdl(rmsnorm_kernel, dim3(M), dim3(kGlueThreads), 0, s, static_cast<const float*>(fp(L.h1)),
-                   static_cast<const float*>(fp(L.dn)), c.h, next_xn, D);
+                   static_cast<const float*>(fp(L.dn)), c.h, next_xn, D, static_cast<uint32_t*>(nullptr));
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

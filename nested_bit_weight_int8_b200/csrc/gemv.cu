@@ -84,6 +84,7 @@ constexpr int kMaxDynSmem = 227 * 1024;
 constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header and alignment slack
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
 constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
+constexpr int kFuseUnitsPerCta = 8; // integer launches up to this many units per CTA skip the prep kernel
 
 // Decode kinds of the planes at one batch row on the integer tensor cores:
 // kDkI8 + r for r = 8, 4, 2. A unit is 256 rows x 128 plane bytes (1024 / r
@@ -134,7 +135,8 @@ struct LinDesc {
   const float* alpha;
   const float* zero;
   float* y;
-  const uint8_t* xf;   // activations in fragment order, n_kc blocks of M*KC bf16
+  const uint8_t* xf;   // activations in fragment order, n_kc blocks of M*KC bf16; in a
+                       // launch without a prep kernel, the input row x itself (bf16)
   const float* psum;   // [M][8] activation sums per class (k >> 1) & 7
   int N, K, r, kc, n_kc, unit_begin;
   int dk;  // decode kind: r for planes, 10 / 11 for the container sliced by Eq. 6 / Eq. 8,
@@ -156,6 +158,9 @@ struct GemvParams {
   uint32_t stage_bytes, off_plane1, off_x;
   int pitch0, pitch1;
   uint32_t* err;
+  // Launches without a prep kernel: grid-barrier words {arrivals, generation}
+  // of the stream, zero between launches.
+  uint32_t* sync;
   unsigned long long wait_ns;
   // 4, 16, 64: left shifts of the integer decode done as multiplies (the FMA
   // pipe) instead of shifts (the ALU pipe, its busiest); as kernel
@@ -509,48 +514,67 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
 }
 
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
-// removes the zero point (once per row, by the part that starts at k-chunk 0)
-// and writes y. The bf16 decode sums x (c - c0), so its zero point is taken
-// relative to the row's centre code: y = A acc - alpha (z - c0 2^(8-r)) Sx;
-// the integer kinds sum x c: y = A acc - alpha z Sx. A row block this CTA
-// owns whole is stored; a shared one is added atomically into y, which the
-// prep kernel zeroed.
+// removes the zero point and writes y. The bf16 decode sums x (c - c0), so
+// its zero point is taken relative to the row's centre code:
+// y = A acc - alpha (z - c0 2^(8-r)) Sx, once per row by the part that starts
+// at k-chunk 0 (Sx from the class sums). The integer kinds sum x c and each
+// part removes its own share, y = A acc - alpha z sxs, with sxs the input sum
+// of the part's units. A row block this CTA owns whole is stored; a shared one
+// is added atomically into y, zeroed first (by the prep kernel, or inside a
+// launch without one).
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
-                           int T, int lane, const float (&tot)[NT][4]) {
+                           int lane, const float (&tot)[Tiling<NT>::TW][NT][4], float sxs) {
+  constexpr int TW = Tiling<NT>::TW;
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
   const int cmax = L.dk == 11 ? (1 << L.r) : (1 << L.r) - 1;
+  // every row's scales first: one memory round trip for the whole flush
+  float av[TW][2], zv[TW][2];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
-    if (n >= L.N) continue;
-    const float a = L.alpha[n], z = L.zero[n];
-    // the same centre code the decode subtracted (make_rowsub)
-    const float c0 = is_i8(L.dk) ? 0.f : static_cast<float>(centre_code(z, L.r, cmax));
-    const float A = a * scale, B = a * (z - c0 * scale);
+  for (int T = 0; T < TW; ++T)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
+      av[T][h] = n < L.N ? L.alpha[n] : 0.f;
+      zv[T][h] = n < L.N ? L.zero[n] : 0.f;
+    }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int m = nt * 8 + 2 * t + e;
-        if (m >= p.M) continue;
-        float v = tot[nt][2 * h + e];
-        if (kc0 == 0) {
-          // Extra Precision: each listed position adds one code step
-          if (L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
-          const float* P = L.psum + m * kClasses;
-          float Sx = 0.f;
+  for (int T = 0; T < TW; ++T) {
 #pragma unroll
-          for (int i = 0; i < kClasses; ++i) Sx += P[i];
-          v = A * v - B * Sx;
-        } else {
-          v = A * v;
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
+      if (n >= L.N) continue;
+      const float a = av[T][h], z = zv[T][h];
+      // the same centre code the decode subtracted (make_rowsub)
+      const float c0 = is_i8(L.dk) ? 0.f : static_cast<float>(centre_code(z, L.r, cmax));
+      const float A = a * scale, B = a * (z - c0 * scale);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int m = nt * 8 + 2 * t + e;
+          if (m >= p.M) continue;
+          float v = tot[T][nt][2 * h + e];
+          if (is_i8(L.dk)) {
+            if (kc0 == 0 && L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
+            v = A * v - B * sxs;
+          } else if (kc0 == 0) {
+            // Extra Precision: each listed position adds one code step
+            if (L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
+            const float* P = L.psum + m * kClasses;
+            float Sx = 0.f;
+#pragma unroll
+            for (int i = 0; i < kClasses; ++i) Sx += P[i];
+            v = A * v - B * Sx;
+          } else {
+            v = A * v;
+          }
+          float* dst = L.y + static_cast<int64_t>(m) * L.N + n;
+          if (whole) *dst = v;
+          else atomicAdd(dst, v);
         }
-        float* dst = L.y + static_cast<int64_t>(m) * L.N + n;
-        if (whole) *dst = v;
-        else atomicAdd(dst, v);
       }
     }
   }
@@ -707,20 +731,20 @@ __device__ __forceinline__ void process_unit_i8(const uint8_t* st0, uint32_t xad
 }
 
 // run_segment for the integer kinds (one batch row). Each unit's header says
-// whether the prep kernel wrote digits (mode 0) or, for inputs that the
+// whether its activation block holds digits (mode 0) or, for inputs that the
 // digits cannot hold exactly, the bf16 fragments of the width's bf16 path
-// (mode 1). Thread (g, t) of a digit unit holds the int32 sums of columns 2t
-// and 2t + 1, digits 2t and 2t + 1 (column 7 is zero): it weighs them by
-// 2^(7 digit - sigma), sigma = 48 - E. A bf16 unit sums x (c - c0) per row;
-// thread t = 0 adds c0 Sxu back (Sxu, the unit's input sum, is in the
-// header). The partials stay in tot[T][0][0] (row g) and tot[T][0][2] (row
-// g + 8) until the row block is flushed.
+// (mode 1), and gives the unit's input sum Sxu, which adds into sxs for the
+// zero-point term. Thread (g, t) of a digit unit holds the int32 sums of
+// columns 2t and 2t + 1, digits 2t and 2t + 1 (column 7 is zero): it weighs
+// them by 2^(7 digit - sigma), sigma = 48 - E. A bf16 unit sums x (c - c0)
+// per row; thread t = 0 adds c0 Sxu back. The partials stay in tot[T][0][0]
+// (row g) and tot[T][0][2] (row g + 8) until the row block is flushed.
 template <int R, int CAP>
 __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const uint8_t* stages,
                                                uint64_t* full, uint64_t* empty, volatile int* s_abort,
                                                int seg, int& s, uint32_t& ph, bool active,
                                                uint32_t zero_addr, int warp, int lane, int l, int rb,
-                                               float (&tot)[2][1][4]) {
+                                               float (&tot)[2][1][4], float& sxs) {
   const int g = lane >> 2, t = lane & 3;
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
@@ -733,6 +757,7 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
       const uint8_t* hdr = st + p.off_x;
       const uint32_t xs = static_cast<uint32_t>(hdr - smem) + kI8Header;  // data, shared offset
       const int mode = reinterpret_cast<const int*>(hdr)[0];
+      sxs += reinterpret_cast<const float*>(hdr)[2];
       if (mode == 0) {
         const int E = reinterpret_cast<const int*>(hdr)[1];
         int ch[2][2][4];
@@ -791,12 +816,180 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
   return true;
 }
 
+// Stages the activation block of one integer-kind unit (one batch row,
+// inputs kc KC .. kc KC + KC - 1 of the row xr, KC = 1024 / R) in shared
+// memory at blk, in the layout the prep kernel writes to global memory: the
+// header (mode, E, Sxu) and either the seven digit slots or, for inputs the
+// digits cannot hold exactly, the width's bf16 fragments. Run by one whole
+// warp. Used by launches without a prep kernel: the producer warp stages each
+// unit while the unit's weight box is in flight.
+template <int R>
+__device__ __forceinline__ void stage_i8_unit(const uint16_t* __restrict__ xr, int K, int kc, uint8_t* blk,
+                                              int lane) {
+  constexpr int KC = 1024 / R, EPT = KC / 32, CPC = 128 / R, J2 = 16 / R / 2;
+  constexpr int kNone = -100000;
+  const int kbase = kc * KC;
+  // (a) the unit's largest exponent E, smallest exponent f, non-finite
+  // inputs and input sum: lane l holds inputs kbase + EPT l .. + EPT - 1
+  // (all inside K or all past it: K % 32 at r = 8, 4 and K % 64 at r = 2)
+  uint32_t xe[EPT / 2];
+#pragma unroll
+  for (int i = 0; i < EPT / 2; ++i) xe[i] = 0u;
+  const int k0 = kbase + lane * EPT;
+  if (k0 < K) {
+    if constexpr (EPT == 16) {
+      const uint4 va = *reinterpret_cast<const uint4*>(xr + k0);
+      const uint4 vb = *reinterpret_cast<const uint4*>(xr + k0 + 8);
+      xe[0] = va.x; xe[1] = va.y; xe[2] = va.z; xe[3] = va.w;
+      xe[4] = vb.x; xe[5] = vb.y; xe[6] = vb.z; xe[7] = vb.w;
+    } else if constexpr (EPT == 8) {
+      const uint4 va = *reinterpret_cast<const uint4*>(xr + k0);
+      xe[0] = va.x; xe[1] = va.y; xe[2] = va.z; xe[3] = va.w;
+    } else {
+      const uint2 va = *reinterpret_cast<const uint2*>(xr + k0);
+      xe[0] = va.x; xe[1] = va.y;
+    }
+  }
+  // (b)'s inputs too, before anything waits on (a): slot group (s, jj, t)
+  // of 16 inputs (MMAs 2 jj, 2 jj + 1 of chunk 4s + t) goes to 4 / J2 lanes,
+  // each writing every (4 / J2)-th digit g
+  constexpr int LPG = 4 / J2;
+  const int grp = lane / LPG, sub = lane % LPG;
+  const int s = grp / (4 * J2), jj = (grp / 4) % J2, t = grp % 4;
+  const int k16 = kbase + (4 * s + t) * CPC + 16 * jj;
+  uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  if (k16 < K) {
+    const uint4 va = *reinterpret_cast<const uint4*>(xr + k16);
+    const uint4 vb = *reinterpret_cast<const uint4*>(xr + k16 + 8);
+    xw[0] = va.x; xw[1] = va.y; xw[2] = va.z; xw[3] = va.w;
+    xw[4] = vb.x; xw[5] = vb.y; xw[6] = vb.z; xw[7] = vb.w;
+  }
+  int emax = kNone, fmin = 1 << 30;
+  bool bad = false;
+  float xsum = 0.f;
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const uint32_t bits = (u & 1) ? (xe[u >> 1] >> 16) : (xe[u >> 1] & 0xFFFFu);
+    const uint32_t ef = (bits >> 7) & 0xFFu, mf = bits & 0x7Fu;
+    if (ef == 0xFFu) bad = true;
+    xsum += __uint_as_float(bits << 16);
+    if (ef == 0u && mf == 0u) continue;
+    const uint32_t m = ef ? (0x80u | mf) : mf;
+    const int f = static_cast<int>(ef ? ef : 1u) - 134;
+    emax = max(emax, f + 31 - __clz(static_cast<int>(m)));
+    fmin = min(fmin, f);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+    fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
+    xsum += __shfl_xor_sync(0xffffffffu, xsum, o);
+  }
+  const int E = emax == kNone ? 0 : emax;
+  if (emax != kNone && (fmin < E - 48 || E > 100 || E < -72)) bad = true;
+  const bool fallback = __any_sync(0xffffffffu, bad);
+  if (!fallback) {
+    // (b) X = |x| 2^(48 - E) (an integer below 2^49) of each input in k-slot
+    // order b, and the signs
+    uint64_t X[16];
+    uint32_t neg = 0u;
+#pragma unroll
+    for (int b = 0; b < 16; ++b) {
+      const int h = b / 8, bb = b % 8;
+      // the input's index among the 16: r = 8 bytes in order; r = 4 codes
+      // 0, 4, 1, 5, 2, 6, 3, 7 of word 2 jj + h; r = 2 codes 4h + (0, 8, 1,
+      // 9, 2, 10, 3, 11) of word jj
+      const int u = R == 8 ? 8 * h + bb
+                  : R == 4 ? 8 * h + ((bb & 1) ? 4 : 0) + (bb >> 1)
+                           : 4 * h + ((bb & 1) ? 8 : 0) + (bb >> 1);
+      const uint32_t bits = (u & 1) ? (xw[u >> 1] >> 16) : (xw[u >> 1] & 0xFFFFu);
+      const uint32_t ef = (bits >> 7) & 0xFFu, mf = bits & 0x7Fu;
+      const uint32_t m = ef ? (0x80u | mf) : mf;
+      const int sh = static_cast<int>(ef ? ef : 1u) - 134 + 48 - E;  // >= 0 wherever m != 0
+      X[b] = m ? (static_cast<uint64_t>(m) << sh) : 0ull;
+      neg |= ((bits >> 15) & 1u) << b;
+    }
+    for (int g = sub; g < kI8Digits; g += LPG) {
+      uint32_t out[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t word = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int b = 4 * w + i;
+          uint32_t d = static_cast<uint32_t>(X[b] >> (7 * g)) & 127u;
+          if ((neg >> b) & 1u) d = (0u - d) & 0xFFu;
+          word |= d << (8 * i);
+        }
+        out[w] = word;
+      }
+      *reinterpret_cast<uint4*>(blk + kI8Header + (((s * J2 + jj) * kI8Digits + g) * 4 + t) * 16) =
+          make_uint4(out[0], out[1], out[2], out[3]);
+    }
+  } else {
+    // (c) the width's bf16 fragments: group q of 8 inputs of chunk 4s + t at
+    // ((s W8 + q) 4 + t) 16, byte planes (r = 8) pairing codes (c0, c2), (c1, c3)
+    constexpr int W8 = 16 / R;
+    for (int gq = lane; gq < KC / 8; gq += 32) {
+      const int sq = gq / (4 * W8), tq = (gq / W8) % 4, q = gq % W8;
+      const int kg = kbase + (4 * sq + tq) * CPC + 8 * q;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (kg < K) v = *reinterpret_cast<const uint4*>(xr + kg);
+      if constexpr (R == 8) {
+        const uint32_t a = __byte_perm(v.x, v.y, 0x5410), b = __byte_perm(v.x, v.y, 0x7632);
+        const uint32_t c = __byte_perm(v.z, v.w, 0x5410), d = __byte_perm(v.z, v.w, 0x7632);
+        v = make_uint4(a, b, c, d);
+      }
+      *reinterpret_cast<uint4*>(blk + kI8Header + ((sq * W8 + q) * 4 + tq) * 16) = v;
+    }
+  }
+  if (lane == 0) {
+    reinterpret_cast<int*>(blk)[0] = fallback ? 1 : 0;
+    reinterpret_cast<int*>(blk)[1] = E;
+    reinterpret_cast<float*>(blk)[2] = xsum;
+  }
+}
+
+// The stream's grid barrier for launches without a prep kernel. Every CTA
+// arrives once, after zeroing the shared row blocks it starts in; the last
+// arrival resets the count and advances the generation. Called by one thread
+// per CTA after its zeroing stores (a CTA barrier orders them before the
+// fence); returns the generation the CTA arrived in.
+__device__ __forceinline__ uint32_t grid_arrive(uint32_t* sync) {
+  __threadfence();
+  const uint32_t gen = *reinterpret_cast<volatile uint32_t*>(sync + 1);
+  const uint32_t old = atomicAdd(sync, 1u);
+  if (old == gridDim.x - 1) {
+    atomicExch(sync, 0u);
+    __threadfence();
+    atomicAdd(sync + 1, 1u);
+  }
+  return gen;
+}
+
+// Waits (at most limit_ns) until every CTA of the grid has arrived: the
+// generation moved past gen. Returns false if it gave up.
+__device__ __forceinline__ bool grid_wait(const uint32_t* sync, uint32_t gen, uint64_t limit_ns) {
+  const volatile uint32_t* g = reinterpret_cast<const volatile uint32_t*>(sync + 1);
+  bool ok = *g != gen;
+  if (!ok && limit_ns > 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!(ok = (*g != gen)) && globaltimer_ns() - t0 <= limit_ns) __nanosleep(64);
+  }
+  __threadfence();
+  return ok;
+}
+
 // I8: a launch whose linears all take the integer kinds (one batch row,
 // planes of width 8, 4, 2): its instantiation holds only their code paths, so
 // the registers of the bf16 decodes do not press on the integer loop.
-template <int NT, int CAP, bool I8 = false>
+// FUSE (with I8): a launch without a prep kernel. The producer warp stages
+// each unit's activation block from x itself, the consumers zero the shared
+// row blocks, and a grid barrier orders that zeroing before any atomic add.
+template <int NT, int CAP, bool I8 = false, bool FUSE = false>
 __global__ void __launch_bounds__(kGemvThreads, (NT <= 2 ? 2 : 1))
 gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
+  static_assert(!FUSE || (I8 && NT == 1), "launches without a prep kernel are integer-only, one batch row");
   using TL = Tiling<NT>;
   extern __shared__ __align__(128) uint8_t smem[];
   // 1024-byte aligned header and stages: the swizzled plane boxes need it
@@ -805,6 +998,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   uint64_t* full = reinterpret_cast<uint64_t*>(base);
   uint64_t* empty = full + kMaxStages;
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
+  volatile uint32_t* s_gen = reinterpret_cast<volatile uint32_t*>(s_abort + 1);  // grid barrier (FUSE)
   uint8_t* zero_block = base + kHeaderBytes - 64;  // 64 zero bytes read by lanes past M
   uint8_t* stages = base + kHeaderBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -826,7 +1020,93 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
 
   const int u0 = p.cta_begin[blockIdx.x];
   const int u1 = p.cta_begin[blockIdx.x + 1];
-  if (u0 >= u1) return;
+  if (u0 >= u1) {
+    if constexpr (FUSE) {
+      // every CTA arrives at the grid barrier, after the previous grid ended
+      if (threadIdx.x == 0) {
+        pdl_wait_primary();
+        grid_arrive(p.sync);
+      }
+    }
+    return;
+  }
+
+  if constexpr (FUSE) {
+    if (warp == kConsumerWarps) {
+      // -------------------------------------------------- producer (FUSE)
+      // Lane 0 requests each unit's weight box (counted in the stage's
+      // transaction bytes, with no arrival); the warp then writes the unit's
+      // activation block from x and lane 0 arrives, which completes the stage
+      // once the box has landed. Weight boxes do not depend on the previous
+      // grid, so the first stages' boxes go out before waiting for it.
+      Cursor c;
+      cursor_init<TL::RPU>(p, u0, c);
+      Cursor pre_c = c;
+      // weights are read once: first out of L2, ahead of code and small data
+      const uint64_t pol = l2_policy_evict_first();
+      auto issue_weights = [&](const Cursor& cc, int s) {
+        uint8_t* st = stages + static_cast<size_t>(s) * p.stage_bytes;
+        const CUtensorMap* tm = p.map_table ? p.map_table + 2 * cc.l : &p.maps[2 * cc.l];
+        mbar_expect_tx(&full[s], TL::RPU * p.pitch0);
+        tma_load_2d_hint(st, tm, cc.kc * p.pitch0, cc.rb * TL::RPU, &full[s], pol);
+      };
+      auto stage_x = [&](const Cursor& cc, int s) {
+        const LinDesc& L = p.lin[cc.l];
+        const uint16_t* xr = reinterpret_cast<const uint16_t*>(L.xf);  // the input row itself
+        uint8_t* blk = stages + static_cast<size_t>(s) * p.stage_bytes + p.off_x;
+        if (cc.dk == kDkI8 + 8) stage_i8_unit<8>(xr, L.K, cc.kc, blk, lane);
+        else if (cc.dk == kDkI8 + 4) stage_i8_unit<4>(xr, L.K, cc.kc, blk, lane);
+        else stage_i8_unit<2>(xr, L.K, cc.kc, blk, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
+      };
+      const int pre = min(S, u1 - u0);
+      if (lane == 0)
+        for (int i = 0; i < pre; ++i) { issue_weights(c, i); cursor_next<TL::RPU>(p, c); }
+      c = pre_c;
+      for (int i = 0; i < pre; ++i) cursor_next<TL::RPU>(p, c);
+      pdl_wait_primary();
+      {
+        // the inputs of this CTA's first units, into L1 ahead of their staging
+        // (after the wait: the previous grid may have written them)
+        Cursor pc = pre_c;
+        const int n_pf = min(u1 - u0, kFuseUnitsPerCta);
+        for (int i = 0; i < n_pf; ++i) {
+          const LinDesc& L = p.lin[pc.l];
+          const int unit_bytes = (1024 / (pc.dk - kDkI8)) * 2;  // KC bf16 inputs
+          const int64_t first = int64_t(pc.kc) * unit_bytes, end = int64_t(L.K) * 2;
+          for (int off = lane * 128; off < unit_bytes && first + off < end; off += 32 * 128)
+            prefetch_l1(L.xf + first + off);
+          cursor_next<TL::RPU>(p, pc);
+        }
+      }
+      for (int i = 0; i < pre; ++i) { stage_x(pre_c, i); cursor_next<TL::RPU>(p, pre_c); }
+      int issued = pre;
+      for (int u = u0 + pre; u < u1; ++u, ++issued) {
+        const int s = issued % S;
+        int st = 0;  // 0: go on, 1: the wait gave up, 2: the consumers stopped
+        if (lane == 0) {
+          if (!mbar_wait_bounded(&empty[s], ((issued / S) - 1) & 1, p.wait_ns)) st = 1;
+          else if (*s_abort) st = 2;
+        }
+        st = __shfl_sync(0xffffffffu, st, 0);
+        if (st != 0) {
+          if (st == 1 && lane == 0) { atomicOr(p.err, kErrWaitEmpty); *s_abort = 1; }
+          break;
+        }
+        if (lane == 0) issue_weights(c, s);
+        stage_x(c, s);
+        cursor_next<TL::RPU>(p, c);
+      }
+      // no bulk copy may be in flight when this warp exits
+      if (lane == 0) {
+        const int first = issued > S ? issued - S : 0;
+        for (int j = first; j < issued; ++j)
+          if (!mbar_wait_bounded(&full[j % S], (j / S) & 1, 1000000000ull)) atomicOr(p.err, kErrDrain);
+      }
+      return;
+    }
+  }
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -839,6 +1119,8 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       Cursor c;
       cursor_init<TL::RPU>(p, u0, c);
       Cursor pre_c = c;
+      // weights are read once: first out of L2, ahead of code and small data
+      const uint64_t pol = l2_policy_evict_first();
       auto issue_weights = [&](const Cursor& cc, int s) {
         int b0, b1;
         plane_widths_dev(cc.dk, b0, b1);
@@ -849,8 +1131,8 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         // One 2-D box per plane (128 rows x the unit's bytes; rows past N and
         // bytes past K read as zero) plus the unit's activation block.
         mbar_arrive_expect_tx(&full[s], box + bytesx);
-        tma_load_2d(st, tm, cc.kc * p.pitch0, cc.rb * TL::RPU, &full[s]);
-        if (b1) tma_load_2d(st + p.off_plane1, tm + 1, cc.kc * p.pitch1, cc.rb * TL::RPU, &full[s]);
+        tma_load_2d_hint(st, tm, cc.kc * p.pitch0, cc.rb * TL::RPU, &full[s], pol);
+        if (b1) tma_load_2d_hint(st + p.off_plane1, tm + 1, cc.kc * p.pitch1, cc.rb * TL::RPU, &full[s], pol);
       };
       auto issue_x = [&](const Cursor& cc, int s) {
         const LinDesc& L = p.lin[cc.l];
@@ -891,8 +1173,22 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   }
 
   // -------------------------------------------------------------- consumers
-  // Class sums and the zeroed outputs come from the prep kernel.
+  // Class sums and the zeroed outputs come from the prep kernel; without one
+  // (FUSE), the consumers zero the row block this CTA starts inside (the CTA
+  // before adds into it too) and arrive at the grid barrier.
   pdl_wait_primary();
+  bool grid_passed = !FUSE;
+  if constexpr (FUSE) {
+    Cursor c0c;
+    cursor_init<TL::RPU>(p, u0, c0c);
+    if (c0c.kc != 0) {
+      const int n = c0c.rb * TL::RPU + static_cast<int>(threadIdx.x);  // one row per consumer thread
+      if (n < c0c.N) p.lin[c0c.l].y[n] = 0.f;
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    if (threadIdx.x == 0) *s_gen = grid_arrive(p.sync);
+    named_bar_sync(1, kConsumerWarps * 32);
+  }
   const int g = lane >> 2, t = lane & 3;
   uint32_t xaddr[NT], xstep[NT];
   const uint32_t zero_addr = static_cast<uint32_t>(zero_block - smem) + t * 16;  // shared offset
@@ -923,13 +1219,21 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       for (int b = 0; b < NT; ++b)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[T][b][i] = 0.f;
+    if (active && lane == 0) {
+      // the row block's scales, read by the flush after the segment's units
+      const LinDesc& L = p.lin[c.l];
+      const int n0 = c.rb * TL::RPU + warp * TL::RPW;
+      prefetch_l1(L.alpha + n0);
+      prefetch_l1(L.zero + n0);
+    }
     bool ok;
+    float sxs = 0.f;  // input sum of the segment's units (integer kinds)
     const Cdec cd = make_cdec(c.dk, c.r);
     if constexpr (I8) {
       switch (c.dk) {
-        case kDkI8 + 8: ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
-        case kDkI8 + 4: ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
-        default: ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot); break;
+        case kDkI8 + 8: ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
+        case kDkI8 + 4: ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
+        default: ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
       }
     } else {
       switch (c.dk) {
@@ -941,15 +1245,15 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
         // the host plans the integer kinds only for one batch row
         case kDkI8 + 8:
-          if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
           else ok = false;
           break;
         case kDkI8 + 4:
-          if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
           else ok = false;
           break;
         case kDkI8 + 2:
-          if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot);
+          if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
           else ok = false;
           break;
         default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
@@ -971,8 +1275,14 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
           }
         }
       }
-#pragma unroll
-      for (int T = 0; T < TL::TW; ++T) flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, T, lane, tot[T]);
+      if (!whole && !grid_passed) {
+        // the first add into a shared row block waits until every CTA has
+        // zeroed its own (at most the wait limit; past it the flag is set)
+        if (lane == 0 && !grid_wait(p.sync, *s_gen, p.wait_ns)) atomicOr(p.err, kErrWaitGrid);
+        __syncwarp();
+        grid_passed = true;
+      }
+      flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot, sxs);
     }
     u += seg;
     c.kc += seg;
@@ -1139,8 +1449,22 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       const int64_t kbase = int64_t(kc) * KC;
       const uint16_t* xr = reinterpret_cast<const uint16_t*>(L.x);  // one batch row
       // (a) E, the smallest exponent f and non-finite inputs over the unit
+      // (b)'s inputs are loaded with (a)'s, before anything waits on them:
+      // lane < 8 J2 takes slot group (s, jj, t), the 16 inputs of MMAs
+      // 2 jj, 2 jj + 1 of chunk 4s + t
+      const int J2 = 16 / r / 2;
+      const int s_b = lane / (4 * J2), jj_b = (lane / 4) % J2, t_b = lane % 4;
+      const int64_t k16 = kbase + int64_t(4 * s_b + t_b) * cpc + 16 * jj_b;
+      uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (lane < 8 * J2 && k16 < L.K) {  // the 16 inputs lie wholly inside or outside K
+        const uint4 va = *reinterpret_cast<const uint4*>(xr + k16);
+        const uint4 vb = *reinterpret_cast<const uint4*>(xr + k16 + 8);
+        xw[0] = va.x; xw[1] = va.y; xw[2] = va.z; xw[3] = va.w;
+        xw[4] = vb.x; xw[5] = vb.y; xw[6] = vb.z; xw[7] = vb.w;
+      }
       int emax = kNone, fmin = 1 << 30;
       bool bad = false;
+      float xsum = 0.f;  // the unit's input sum (the zero-point term)
       const int ept = KC / 32;  // 4, 8 or 16 consecutive inputs per lane (all in or all out: K % 32
                                 // at r = 8 and 4, K % 64 at r = 2)
       const int64_t k0 = kbase + int64_t(lane) * ept;
@@ -1164,6 +1488,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
         const uint32_t bits = (u & 1) ? (xe[u >> 1] >> 16) : (xe[u >> 1] & 0xFFFFu);
         const uint32_t ef = (bits >> 7) & 0xFFu, mf = bits & 0x7Fu;
         if (ef == 0xFFu) bad = true;
+        xsum += __uint_as_float(bits << 16);
         if (ef == 0u && mf == 0u) continue;
         const uint32_t m = ef ? (0x80u | mf) : mf;
         const int f = static_cast<int>(ef ? ef : 1u) - 134;
@@ -1174,6 +1499,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       for (int o = 16; o > 0; o >>= 1) {
         emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
         fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
+        xsum += __shfl_xor_sync(0xffffffffu, xsum, o);
       }
       const int E = emax == kNone ? 0 : emax;
       if (emax != kNone && (fmin < E - 48 || E > 100 || E < -72)) bad = true;
@@ -1183,18 +1509,9 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
       if (!fallback) {
         // (b) digit g of slot group (s, jj, t): MMAs j = 2 jj, 2 jj + 1 of chunk
         // 4s + t, whose 16 inputs are the chunk's codes 16 jj .. 16 jj + 15
-        // (loaded at once), in the k-slot order of i8_regs
-        const int J2 = 16 / r / 2;
+        // (loaded above), in the k-slot order of i8_regs
         if (lane < 8 * J2) {
-          const int s = lane / (4 * J2), jj = (lane / 4) % J2, t = lane % 4;
-          const int64_t k16 = kbase + int64_t(4 * s + t) * cpc + 16 * jj;
-          uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          if (k16 < L.K) {  // the 16 inputs lie wholly inside or outside K (K % 32 == 0)
-            const uint4 va = *reinterpret_cast<const uint4*>(xr + k16);
-            const uint4 vb = *reinterpret_cast<const uint4*>(xr + k16 + 8);
-            xw[0] = va.x; xw[1] = va.y; xw[2] = va.z; xw[3] = va.w;
-            xw[4] = vb.x; xw[5] = vb.y; xw[6] = vb.z; xw[7] = vb.w;
-          }
+          const int s = s_b, jj = jj_b, t = t_b;
           uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
           for (int b = 0; b < 16; ++b) {
@@ -1223,7 +1540,7 @@ __global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ 
         if (g == 0 && lane == 0) {
           reinterpret_cast<int*>(blk)[0] = 0;
           reinterpret_cast<int*>(blk)[1] = E;
-          reinterpret_cast<float*>(blk)[2] = 0.f;
+          reinterpret_cast<float*>(blk)[2] = xsum;
         }
       } else if (g == 0) {
         // (c) the width's bf16 fragments: group q of 8 inputs of chunk 4s + t at
@@ -1310,9 +1627,9 @@ std::mutex g_cache_mutex;
 
 // Persistent grid for `units` work units at `smem` bytes of shared memory:
 // every resident CTA slot of the device, at most one CTA per unit.
-template <int NT, int CAP, bool I8 = false>
+template <int NT, int CAP, bool I8 = false, bool FUSE = false>
 cudaError_t gemv_grid(size_t smem, int sms, int units, int* grid_out) {
-  auto kern = gemv_streamk_kernel<NT, CAP, I8>;
+  auto kern = gemv_streamk_kernel<NT, CAP, I8, FUSE>;
   static std::map<int, KernelCache> caches;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1340,9 +1657,9 @@ cudaError_t gemv_grid(size_t smem, int sms, int units, int* grid_out) {
   return cudaSuccess;
 }
 
-template <int NT, int CAP, bool I8 = false>
+template <int NT, int CAP, bool I8 = false, bool FUSE = false>
 cudaError_t launch_gemv(const GemvParams<CAP>& gp, size_t smem, int grid, cudaStream_t stream) {
-  auto kern = gemv_streamk_kernel<NT, CAP, I8>;
+  auto kern = gemv_streamk_kernel<NT, CAP, I8, FUSE>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -1594,21 +1911,61 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     if (++n_ep > kMaxEpJobs) return cudaErrorNotSupported;
     ep_off += (size_t(M) * jobs[i].N * sizeof(float) + 255) & ~size_t(255);
   }
-  const size_t ws_bytes = ep_off + 256;
-  void* ws = nullptr;
+  // Stage layout: [128 rows x P0][128 rows x P1][M x KC bf16 activations].
+  const int P1 = two_planes ? P0 / 2 : 0;
+  const uint32_t off_plane1 = static_cast<uint32_t>(RU * P0);
+  const uint32_t off_x = off_plane1 + static_cast<uint32_t>(RU * P1);
+  uint32_t stage_bytes = off_x + x_unit_max;
+  stage_bytes = (stage_bytes + 1023) & ~1023u;  // swizzled boxes start 1024-aligned
+  int stages = static_cast<int>(kStageBudget / stage_bytes);
+  stages = std::max(2, std::min(stages, kMaxStages));
+  const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(stages) * stage_bytes;
+  const int sms = sm_count();
+  bool i8_only = true;
+  for (int i = 0; i < n_jobs; ++i) i8_only = i8_only && is_i8(gp.lin[i].dk);
   cudaError_t e = cudaSuccess;
+  int grid = 1;
+  // A short integer launch (at most kFuseUnitsPerCta units per CTA) runs
+  // without the prep kernel: its producer warps stage the activation blocks
+  // themselves, which takes the prep grid and its wait off the call's path.
+  // Longer launches keep the prep kernel, which stages every block once.
+  bool fuse = false;
+  if (NT == 1 && i8_only && n_ep == 0 && (!fixed || fixed->sync)) {
+    e = gemv_grid<1, CAP, true, true>(smem, sms, units, &grid);
+    if (e != cudaSuccess) return e;
+    fuse = int64_t(units) <= int64_t(kFuseUnitsPerCta) * grid;
+  }
+  if (!fuse) {
+    switch (NT) {
+      case 1: e = i8_only ? gemv_grid<1, CAP, true>(smem, sms, units, &grid) : gemv_grid<1, CAP>(smem, sms, units, &grid); break;
+      case 2: e = gemv_grid<2, CAP>(smem, sms, units, &grid); break;
+      case 3: e = gemv_grid<3, CAP>(smem, sms, units, &grid); break;
+      default: e = gemv_grid<4, CAP>(smem, sms, units, &grid); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+
+  const size_t ws_bytes = fuse ? 0 : ep_off + 256;
+  void* ws = nullptr;
+  uint32_t* sync = nullptr;
   if (fixed) {
     if (ws_bytes > fixed->bytes) return cudaErrorMemoryAllocation;
     ws = fixed->ptr;
+    sync = fixed->sync;
   } else {
-    e = get_workspace(stream, ws_bytes, &ws);
+    e = get_workspace(stream, ws_bytes, &ws, &sync);
     if (e != cudaSuccess) return e;
   }
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* psum_base = reinterpret_cast<float*>(wsb + psum_off);
   for (int i = 0; i < n_jobs; ++i) {
-    gp.lin[i].xf = wsb + layouts[lay_of[i]].off;
-    gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * kClasses;
+    if (fuse) {
+      gp.lin[i].xf = static_cast<const uint8_t*>(jobs[i].x);  // the producers read x itself
+      gp.lin[i].psum = nullptr;
+    } else {
+      gp.lin[i].xf = wsb + layouts[lay_of[i]].off;
+      gp.lin[i].psum = psum_base + size_t(sum_of[i]) * M * kClasses;
+    }
   }
   {
     size_t off = ep_begin;
@@ -1624,27 +1981,6 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     }
     pp.n_ep = k;
   }
-
-  // Stage layout: [128 rows x P0][128 rows x P1][M x KC bf16 activations].
-  const int P1 = two_planes ? P0 / 2 : 0;
-  const uint32_t off_plane1 = static_cast<uint32_t>(RU * P0);
-  const uint32_t off_x = off_plane1 + static_cast<uint32_t>(RU * P1);
-  uint32_t stage_bytes = off_x + x_unit_max;
-  stage_bytes = (stage_bytes + 1023) & ~1023u;  // swizzled boxes start 1024-aligned
-  int stages = static_cast<int>(kStageBudget / stage_bytes);
-  stages = std::max(2, std::min(stages, kMaxStages));
-  const size_t smem = 1024 /* alignment slack */ + kHeaderBytes + size_t(stages) * stage_bytes;
-  const int sms = sm_count();
-  bool i8_only = true;
-  for (int i = 0; i < n_jobs; ++i) i8_only = i8_only && is_i8(gp.lin[i].dk);
-  int grid = 1;
-  switch (NT) {
-    case 1: e = i8_only ? gemv_grid<1, CAP, true>(smem, sms, units, &grid) : gemv_grid<1, CAP>(smem, sms, units, &grid); break;
-    case 2: e = gemv_grid<2, CAP>(smem, sms, units, &grid); break;
-    case 3: e = gemv_grid<3, CAP>(smem, sms, units, &grid); break;
-    default: e = gemv_grid<4, CAP>(smem, sms, units, &grid); break;
-  }
-  if (e != cudaSuccess) return e;
 
   // CTA ranges of equal estimated cost, and the row blocks they share.
   int64_t total_cost = 0;
@@ -1713,13 +2049,15 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
     pp.sum[i] = {static_cast<const __nv_bfloat16*>(sum_x[i]),
                  psum_base + size_t(i) * M * kClasses, sum_k[i]};
   }
-  int prep_grid = std::max(n_sums * M, sms);
-  if (pp.n_ep > 0) prep_grid = 4 * sms;  // the Extra Precision gathers want many warps in flight
-  // one warp per (unit, digit) of the digit layouts, all in one round
-  prep_grid = std::max(prep_grid, (pp.n_i8 * kI8Digits + 7) / 8);
-  prep_grid = std::min(prep_grid, 4 * sms);
-  e = launch_pdl(gemv_prep_kernel<CAP>, dim3(prep_grid), dim3(256), 0, stream, pp);
-  if (e != cudaSuccess) return e;
+  if (!fuse) {
+    int prep_grid = std::max(n_sums * M, sms);
+    if (pp.n_ep > 0) prep_grid = 4 * sms;  // the Extra Precision gathers want many warps in flight
+    // one warp per (unit, digit) of the digit layouts, all in one round
+    prep_grid = std::max(prep_grid, (pp.n_i8 * kI8Digits + 7) / 8);
+    prep_grid = std::min(prep_grid, 4 * sms);
+    e = launch_pdl(gemv_prep_kernel<CAP>, dim3(prep_grid), dim3(256), 0, stream, pp);
+    if (e != cudaSuccess) return e;
+  }
 
   gp.n_lin = n_jobs;
   gp.M = M;
@@ -1731,11 +2069,13 @@ cudaError_t run_gemv_cap(const LinearJob* jobs, int n_jobs, int M, cudaStream_t 
   gp.pitch0 = P0;
   gp.pitch1 = P1;
   gp.err = err;
+  gp.sync = sync;
   gp.wait_ns = wait_limit_ns();
   gp.shl[0] = 4u;
   gp.shl[1] = 16u;
   gp.shl[2] = 64u;
 
+  if (fuse) return launch_gemv<1, CAP, true, true>(gp, smem, grid, stream);
   switch (NT) {
     case 1: return i8_only ? launch_gemv<1, CAP, true>(gp, smem, grid, stream) : launch_gemv<1, CAP>(gp, smem, grid, stream);
     case 2: return launch_gemv<2, CAP>(gp, smem, grid, stream);

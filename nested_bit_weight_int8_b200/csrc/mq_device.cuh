@@ -14,6 +14,7 @@ constexpr uint32_t kErrWaitEmpty = 2u;     // producer waited too long for a fre
 constexpr uint32_t kErrDrain = 4u;         // copies still in flight at exit
 constexpr uint32_t kErrMma = 8u;           // tensor-core pipeline wait gave up
 constexpr uint32_t kErrBounds = 16u;       // a debug build's index check failed
+constexpr uint32_t kErrWaitGrid = 32u;     // a CTA waited too long at a grid-wide barrier
 
 // Index checks of the debug build (compiled with MQ_DEBUG_BOUNDS): a check
 // that fails sets kErrBounds in the error word and the guarded access is
@@ -58,6 +59,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
+               : "memory");
+}
+
+// Raises the transaction count of the current phase by `bytes` without an
+// arrival (the arrival comes separately, e.g. after threads wrote shared
+// memory that the same phase publishes).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
 
@@ -125,6 +134,30 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, in
       : "memory");
 }
 
+// An L2 policy that marks lines as the first to evict: for data read once and
+// streamed through (decode weights), so that it does not push out what later
+// calls read again (instructions, activations, scales, outputs).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_2d with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const void* tmap, int c0, int c1,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Requests the line holding `p` into L1 ahead of a later load.
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
@@ -135,6 +168,11 @@ __device__ __forceinline__ void pdl_wait_primary() {
 }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier over the first `threads` threads of the CTA (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // ---------------------------------------------------------------- MMA

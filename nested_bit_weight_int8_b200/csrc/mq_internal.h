@@ -82,8 +82,12 @@ struct Workspace {
   size_t bytes = 0;
 };
 // Returns a workspace of at least `bytes` for the current device and
-// `stream`, growing it if needed (growth synchronizes the device).
-cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out);
+// `stream`, growing it if needed (growth synchronizes the device). Each
+// workspace starts with kSyncBytes of grid-barrier words, zeroed when it is
+// allocated, that the decode launches without a prep kernel use: `sync` (if
+// not null) receives their address, `out` the bytes after them.
+constexpr size_t kSyncBytes = 256;
+cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out, uint32_t** sync = nullptr);
 // Device error word of the current device (zero-initialized).
 cudaError_t get_error_word(uint32_t** out);
 uint64_t wait_limit_ns();
@@ -121,6 +125,7 @@ struct FixedScratch {
   void* ptr;
   size_t bytes;
   uint32_t* err;
+  uint32_t* sync;  // grid-barrier words (zero-initialized)
 };
 // Reads and clears the wait-error word of mq_linear_noalloc's fixed array on
 // the current device (0 if that entry point never ran there).

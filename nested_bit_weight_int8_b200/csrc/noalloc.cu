@@ -119,7 +119,8 @@ extern "C" mq_status mq_linear_noalloc(const void* x, int64_t M, int64_t K, cons
   cudaError_t e = noalloc_base(&base);
   if (e != cudaSuccess) return noalloc_fail(MQ_ERR_CUDA, "mq_linear_noalloc: set-up: %s", cudaGetErrorString(e));
   unsigned char* b = static_cast<unsigned char*>(base);
-  FixedScratch fs{b + kNoAllocHeader, have, reinterpret_cast<uint32_t*>(b)};
+  // header: the error word at byte 0, the grid-barrier words at byte 128
+  FixedScratch fs{b + kNoAllocHeader, have, reinterpret_cast<uint32_t*>(b), reinterpret_cast<uint32_t*>(b + 128)};
   e = run_gemv_fixed(job, static_cast<int>(M), static_cast<cudaStream_t>(stream), fs);
   if (e != cudaSuccess) return noalloc_fail(MQ_ERR_CUDA, "mq_linear_noalloc: %s", cudaGetErrorString(e));
   return MQ_OK;
