@@ -79,7 +79,12 @@ namespace {
 constexpr int kConsumerWarps = 8;
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxStages = 8;
-constexpr int kHeaderBytes = 1024;  // barriers, abort flag; last 64 bytes: zero block
+// Header: barriers and flags from byte 0, a 64-byte zero block ending at
+// byte 1024, then each consumer warp's row scales (alpha and z of its 32
+// rows, 256 bytes a warp) up to byte 3072, where the stages start.
+constexpr int kHeaderBytes = 3072;
+constexpr int kScalesOff = 1024;
+static_assert(kScalesOff + kConsumerWarps * 64 * 4 <= kHeaderBytes, "row scales overflow the header");
 constexpr int kMaxDynSmem = 227 * 1024;
 constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header and alignment slack
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
@@ -247,10 +252,10 @@ struct RowSub {
 };
 
 template <int R>
-__device__ __forceinline__ RowSub make_rowsub(const float* zero, int n, int N, int r) {
+__device__ __forceinline__ RowSub make_rowsub(float zero, int r) {
   const int rw = (R == 10 || R == 11) ? r : R;
   const int cmax = R == 11 ? (1 << rw) : (1 << rw) - 1;
-  const int c0 = n < N ? centre_code(zero[n], rw, cmax) : 0;
+  const int c0 = centre_code(zero, rw, cmax);  // rows past N: z = 0, c0 = 0
   // the low plane's magics: r = 2 by bit position 1, 3, 5; r = 3 by 3, 5;
   // r = 4 and 6 one; the container the power of two 2^r (Eq. 6) or 2^(r+1)
   const int m0 = R == 2 ? 64 : (R == 3 || R == 4 || R == 6) ? 16 : (R == 10 ? (1 << rw) : (2 << rw));
@@ -513,6 +518,22 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
   }
 }
 
+// Copies alpha and z of this warp's rows of row block rb of linear l into
+// its shared slots sc[0..31] (alpha) and sc[32..63] (z), asynchronously
+// (cp.async, waited for before their first use); rows past N read as zero.
+// The scales do not change during a launch, so the first copy is issued
+// before the wait for the previous grid.
+template <int NT, int CAP>
+__device__ __forceinline__ void stage_scales(const GemvParams<CAP>& p, int l, int rb, int warp, int lane,
+                                             float* sc) {
+  const LinDesc& L = p.lin[l];
+  const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + lane;
+  const bool in = lane < Tiling<NT>::RPW && n < L.N;
+  cp_async_4(sc + lane, in ? L.alpha + n : L.alpha, in ? 4u : 0u);
+  cp_async_4(sc + 32 + lane, in ? L.zero + n : L.zero, in ? 4u : 0u);
+  cp_async_commit();
+}
+
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
 // removes the zero point and writes y. The bf16 decode sums x (c - c0), so
 // its zero point is taken relative to the row's centre code:
@@ -524,21 +545,21 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
 // launch without one).
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
-                           int lane, const float (&tot)[Tiling<NT>::TW][NT][4], float sxs) {
+                           int lane, const float (&tot)[Tiling<NT>::TW][NT][4], float sxs, const float* sc) {
   constexpr int TW = Tiling<NT>::TW;
   const LinDesc& L = p.lin[l];
   const int g = lane >> 2, t = lane & 3;
   const float scale = static_cast<float>(1 << (8 - L.r));
   const int cmax = L.dk == 11 ? (1 << L.r) : (1 << L.r) - 1;
-  // every row's scales first: one memory round trip for the whole flush
+  // the row scales, staged in shared memory (stage_scales)
   float av[TW][2], zv[TW][2];
 #pragma unroll
   for (int T = 0; T < TW; ++T)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
-      av[T][h] = n < L.N ? L.alpha[n] : 0.f;
-      zv[T][h] = n < L.N ? L.zero[n] : 0.f;
+      const int i = 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
+      av[T][h] = sc[i];
+      zv[T][h] = sc[32 + i];
     }
 #pragma unroll
   for (int T = 0; T < TW; ++T) {
@@ -591,18 +612,21 @@ __device__ __forceinline__ bool run_segment(const GemvParams<CAP>& p, const uint
                                             bool active, const uint32_t (&xaddr)[NT],
                                             const uint32_t (&xstep)[NT], int warp, int lane,
                                             const Cdec& cd, int l, int rb,
-                                            float (&tot)[Tiling<NT>::TW][NT][4]) {
+                                            float (&tot)[Tiling<NT>::TW][NT][4], const float* sc) {
   constexpr int TW = Tiling<NT>::TW;
-  // the centre codes of this thread's rows (rows g and g + 8 of each tile)
+  // the centre codes of this thread's rows (rows g and g + 8 of each tile),
+  // from the row scales staged in shared memory
   RowSub rs[TW][2];
   {
     const LinDesc& L = p.lin[l];
     const int g = lane >> 2;
+    cp_async_wait_all();
+    __syncwarp();
 #pragma unroll
     for (int T = 0; T < TW; ++T)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h, L.N, L.r);
+        rs[T][h] = make_rowsub<R>(sc[32 + 16 * T + Tiling<NT>::frag_row(g) + 8 * h], L.r);
   }
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
@@ -744,7 +768,7 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
                                                uint64_t* full, uint64_t* empty, volatile int* s_abort,
                                                int seg, int& s, uint32_t& ph, bool active,
                                                uint32_t zero_addr, int warp, int lane, int l, int rb,
-                                               float (&tot)[2][1][4], float& sxs) {
+                                               float (&tot)[2][1][4], float& sxs, const float* sc) {
   const int g = lane >> 2, t = lane & 3;
   for (int i = 0; i < seg; ++i) {
     if (*s_abort || !mbar_wait_bounded(&full[s], ph, p.wait_ns)) {
@@ -795,11 +819,13 @@ __device__ __forceinline__ bool run_segment_i8(const GemvParams<CAP>& p, const u
         // rather than held in registers across the unit loop
         RowSub rs[2][2];
         const LinDesc& L = p.lin[l];
+        cp_async_wait_all();
+        __syncwarp();
 #pragma unroll
         for (int T = 0; T < 2; ++T)
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            rs[T][h] = make_rowsub<R>(L.zero, rb * Tiling<1>::RPU + warp * Tiling<1>::RPW + 16 * T + Tiling<1>::frag_row(g) + 8 * h, L.N, L.r);
+            rs[T][h] = make_rowsub<R>(sc[32 + 16 * T + Tiling<1>::frag_row(g) + 8 * h], L.r);
         process_unit<R, 1>(st, st + Tiling<1>::RPU * Tiling<1>::P0, xa, xstep, warp, lane, Cdec{0u, 0u, 0u},
                            rs, p.err, ch);
 #pragma unroll
@@ -999,7 +1025,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   uint64_t* empty = full + kMaxStages;
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
   volatile uint32_t* s_gen = reinterpret_cast<volatile uint32_t*>(s_abort + 1);  // grid barrier (FUSE)
-  uint8_t* zero_block = base + kHeaderBytes - 64;  // 64 zero bytes read by lanes past M
+  uint8_t* zero_block = base + kScalesOff - 64;  // 64 zero bytes read by lanes past M
   uint8_t* stages = base + kHeaderBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
@@ -1173,6 +1199,14 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   }
 
   // -------------------------------------------------------------- consumers
+  // This warp's row scales slots; the first segment's copy goes out before
+  // the wait for the previous grid (the scales are constant).
+  float* sc = reinterpret_cast<float*>(base + kScalesOff) + warp * 64;
+  {
+    Cursor c1;
+    cursor_init<TL::RPU>(p, u0, c1);
+    stage_scales<NT>(p, c1.l, c1.rb, warp, lane, sc);
+  }
   // Class sums and the zeroed outputs come from the prep kernel; without one
   // (FUSE), the consumers zero the row block this CTA starts inside (the CTA
   // before adds into it too) and arrive at the grid barrier.
@@ -1206,8 +1240,16 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   cursor_init<TL::RPU>(p, u0, c);
   int s = 0;
   uint32_t ph = 0;
+  bool first_seg = true;
   for (int u = u0; u < u1;) {
     // One row block: units kc0 .. kc0 + seg - 1 of (linear c.l, row block c.rb).
+    if (!first_seg) {
+      // the previous copy has landed (and the flush read it) before the slots are reused
+      cp_async_wait_all();
+      __syncwarp();
+      stage_scales<NT>(p, c.l, c.rb, warp, lane, sc);
+    }
+    first_seg = false;
     const int seg = min(c.n_kc - c.kc, u1 - u);
     const int kc0 = c.kc;
     const bool whole = kc0 == 0 && seg == c.n_kc;
@@ -1219,44 +1261,37 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       for (int b = 0; b < NT; ++b)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[T][b][i] = 0.f;
-    if (active && lane == 0) {
-      // the row block's scales, read by the flush after the segment's units
-      const LinDesc& L = p.lin[c.l];
-      const int n0 = c.rb * TL::RPU + warp * TL::RPW;
-      prefetch_l1(L.alpha + n0);
-      prefetch_l1(L.zero + n0);
-    }
     bool ok;
     float sxs = 0.f;  // input sum of the segment's units (integer kinds)
     const Cdec cd = make_cdec(c.dk, c.r);
     if constexpr (I8) {
       switch (c.dk) {
-        case kDkI8 + 8: ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
-        case kDkI8 + 4: ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
-        default: ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs); break;
+        case kDkI8 + 8: ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc); break;
+        case kDkI8 + 4: ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc); break;
+        default: ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc); break;
       }
     } else {
       switch (c.dk) {
-        case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
-        case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
-        case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
-        case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
-        case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
-        case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        case 2: ok = run_segment<2, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
+        case 4: ok = run_segment<4, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
+        case 8: ok = run_segment<8, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
+        case 3: ok = run_segment<3, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
+        case 10: ok = run_segment<10, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
+        case 11: ok = run_segment<11, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
         // the host plans the integer kinds only for one batch row
         case kDkI8 + 8:
-          if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
+          if constexpr (NT == 1) ok = run_segment_i8<8>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc);
           else ok = false;
           break;
         case kDkI8 + 4:
-          if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
+          if constexpr (NT == 1) ok = run_segment_i8<4>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc);
           else ok = false;
           break;
         case kDkI8 + 2:
-          if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs);
+          if constexpr (NT == 1) ok = run_segment_i8<2>(p, stages, full, empty, s_abort, seg, s, ph, active, zero_addr, warp, lane, c.l, c.rb, tot, sxs, sc);
           else ok = false;
           break;
-        default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot); break;
+        default: ok = run_segment<6, NT>(p, stages, full, empty, s_abort, seg, s, ph, active, xaddr, xstep, warp, lane, cd, c.l, c.rb, tot, sc); break;
       }
     }
     if (!ok) break;  // outputs are undefined after a give-up; the flag says so
@@ -1282,7 +1317,9 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
         __syncwarp();
         grid_passed = true;
       }
-      flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot, sxs);
+      cp_async_wait_all();  // the row scales (bf16 segments waited already)
+      __syncwarp();
+      flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot, sxs, sc);
     }
     u += seg;
     c.kc += seg;
@@ -1294,6 +1331,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       }
     }
   }
+  cp_async_wait_all();  // no copy into shared memory outlives the thread
 }
 
 // ------------------------------------------------------------------ prep
