@@ -199,12 +199,15 @@ MQ_API mq_status mq_ep_overflow_cols(const uint8_t* q, int64_t N, int64_t K, int
 /*
  * The Extra Precision product from the Eq. 6 planes plus the sparse list:
  *   y[m,n] = sum_k x[m,k] alpha_n (code8[n,k] 2^s - z_n),
- * code8 the unclamped Eq. 8 code, computed as the planes' product plus
- * alpha_n 2^s sum over row n's listed positions of x[m,k] (the "sparse
- * additions"), fused into the decode kernel's epilogue. Arguments as
- * mq_linear plus the list of mq_ep_overflow_*; requires 1 <= M <= 32 (larger
- * M returns MQ_ERR_UNSUPPORTED), r in {6, 4, 3, 2}, K <= 65536. Accuracy as
- * mq_linear, against W with the Eq. 8 codes.
+ * code8 the unclamped Eq. 8 code. At M <= 32 (decode) it is the planes'
+ * product plus alpha_n 2^s times the sum over row n's listed positions of
+ * x[m,k] (the "sparse additions"), gathered by the prep kernel and added in
+ * the decode epilogue. At M > 32 (prefill) the list is first laid out as a
+ * bit plane (N x K/32 words in the library's workspace) and the GEMM's
+ * decode adds one step to each listed code before the tensor cores sum
+ * x (code8 - c0). Arguments as mq_linear plus the list of mq_ep_overflow_*;
+ * r in {6, 4, 3, 2}, K <= 65536. Accuracy as mq_linear, against W with the
+ * Eq. 8 codes.
  */
 MQ_API mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed,
                               const float* alpha, const float* zero, int64_t N, int r,

@@ -303,9 +303,16 @@ mq_status mq_linear_ep(const void* x, int64_t M, int64_t K, const void* packed, 
   if (!row_ptr || !cols || !aligned(row_ptr, 4) || !aligned(cols, 2))
     return fail(MQ_ERR_INVALID_ARG, "mq_linear_ep: row_ptr / cols null or misaligned");
   if (K > 65536) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: K > 65536");
-  if (M > 32) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: M must be <= 32 (decode path)");
   LinearJob job{x, static_cast<const uint8_t*>(packed), alpha, zero, y, N, K, r, kPlanes, row_ptr, cols};
-  cudaError_t e = run_gemv(&job, 1, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M <= 32) {
+    e = run_gemv(&job, 1, static_cast<int>(M), s);
+  } else {
+    if (M > (int64_t(1) << 24)) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: M too large");
+    e = run_gemm(job, static_cast<int>(M), s);
+  }
+  if (e == cudaErrorNotSupported) return fail(MQ_ERR_UNSUPPORTED, "mq_linear_ep: shape not served by this build");
   if (e != cudaSuccess) return cuda_fail(e, "mq_linear_ep");
   return MQ_OK;
 }

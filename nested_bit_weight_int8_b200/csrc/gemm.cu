@@ -69,6 +69,10 @@ struct GemmParams {
   int M, N, K, r;
   uint32_t stage_bytes;    // x sub-tiles + plane 0 box + plane 1 box, 1024-aligned
   uint32_t off_p0, off_p1; // plane boxes within a stage
+  // Extra Precision (Eq. 8): the listed positions as a bit plane, row n's
+  // bit k at word n * ep_words + k / 32, bit k % 32 (null without a list)
+  const uint32_t* ep_bits;
+  int ep_words;
 };
 
 // ------------------------------------------------------------ Sx kernel
@@ -130,10 +134,14 @@ __device__ __forceinline__ uint32_t exact_pair_bytes(uint32_t w, uint32_t sel_lo
 // width r): code = min(q + 2^(s-1), 255) >> s, or (q + 2^(s-1)) >> s, on the
 // two 16-bit halves at once (h2 = 2^(s-1) in both halves, kmask the code's
 // bits in both halves after the shift by s).
+// epw (planes of width 2, 3, 4, 6): the Extra Precision steps of the 32
+// codes, bit j for code 2j and bit 16 + j for code 2j + 1; each set bit adds
+// one to its code (the Eq. 8 code is the Eq. 6 code plus one there, at most
+// 2^r <= 64, still under the magic 128).
 template <int R>
 __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, const uint8_t* p1,
                                          uint32_t (&v)[16], uint32_t sub2, float subf, uint32_t h2 = 0,
-                                         uint32_t kmask = 0, int sh = 0) {
+                                         uint32_t kmask = 0, int sh = 0, uint32_t epw = 0) {
   if constexpr (R == 10 || R == 11) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint4 b = *reinterpret_cast<const uint4*>(p0b);
@@ -149,12 +157,14 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     const uint2 a = *reinterpret_cast<const uint2*>(p0);
     const uint32_t w[2] = {a.x, a.y};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 8] >> (2 * (j % 8))) & 0x00030003u, sub2);
+    for (int j = 0; j < 16; ++j)
+      v[j] = exact_pair(((w[j / 8] >> (2 * (j % 8))) & 0x00030003u) + ((epw >> j) & 0x00010001u), sub2);
   } else if constexpr (R == 4) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = exact_pair((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu, sub2);
+    for (int j = 0; j < 16; ++j)
+      v[j] = exact_pair(((w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu) + ((epw >> j) & 0x00010001u), sub2);
   } else if constexpr (R == 3) {
     const uint2 a = *reinterpret_cast<const uint2*>(p0);
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p1);
@@ -163,7 +173,7 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     for (int j = 0; j < 16; ++j) {
       const uint32_t lo = (w[j / 8] >> (2 * (j % 8))) & 0x00030003u;
       const uint32_t hi = ((u >> j) & 0x00010001u) << 2;
-      v[j] = exact_pair(lo | hi, sub2);
+      v[j] = exact_pair((lo | hi) + ((epw >> j) & 0x00010001u), sub2);
     }
   } else if constexpr (R == 6) {
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
@@ -174,7 +184,7 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
     for (int j = 0; j < 16; ++j) {
       const uint32_t lo = (w[j / 4] >> (4 * (j % 4))) & 0x000F000Fu;
       const uint32_t hi = ((u[j / 8] >> (2 * (j % 8))) & 0x00030003u) << 4;
-      v[j] = exact_pair(lo | hi, sub2);
+      v[j] = exact_pair((lo | hi) + ((epw >> j) & 0x00010001u), sub2);
     }
   } else {  // R == 8: bytes, 4 codes per word
     const uint4 a = *reinterpret_cast<const uint4*>(p0);
@@ -187,10 +197,26 @@ __device__ __forceinline__ void decode32(const uint8_t* p0, const uint8_t* p0b, 
   }
 }
 
+// The 32 position bits m of a half stage (bit i: code i) rearranged for
+// decode32: the even codes' bits to bits 0..15, the odd codes' to 16..31.
+__device__ __forceinline__ uint32_t spread_even_odd(uint32_t m) {
+  auto compact = [](uint32_t e) {  // bits 0, 2, 4, ... of e to bits 0, 1, 2, ...
+    e &= 0x55555555u;
+    e = (e | (e >> 1)) & 0x33333333u;
+    e = (e | (e >> 2)) & 0x0F0F0F0Fu;
+    e = (e | (e >> 4)) & 0x00FF00FFu;
+    e = (e | (e >> 8)) & 0x0000FFFFu;
+    return e;
+  };
+  return compact(m) | (compact(m >> 1) << 16);
+}
+
 // ------------------------------------------------------------ kernel
-template <int R>
+// EP: the planes carry an Extra Precision bit plane (widths 2, 3, 4, 6).
+template <int R, bool EP = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
+  static_assert(!EP || R == 2 || R == 3 || R == 4 || R == 6, "Extra Precision needs planes of width <= 6");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base: the swizzled x sub-tiles need it.
   const uint32_t raw = smem_u32(smem_raw);
@@ -325,6 +351,14 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
     bool ok = true;
     for (int it = grp; it < n_k; it += 2) {
       const int s = it % kStages;
+      // this row's Extra Precision steps in the warp's 32 codes of the stage
+      // (the bit plane is ready before the launch, so it loads ahead of the wait)
+      uint32_t epw = 0;
+      if constexpr (EP) {
+        const int kw = (it * kBK + 32 * h) >> 5;
+        if (n0 + row < p.N && kw < p.ep_words)
+          epw = spread_even_odd(__ldg(p.ep_bits + static_cast<int64_t>(n0 + row) * p.ep_words + kw));
+      }
       // Every lane waits (each needs the barrier's ordering for the staged
       // bytes); the warp then decides together, since the tensor-memory
       // store below must be executed by all of its lanes.
@@ -363,7 +397,7 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
       (void)st_end;  // read only by the debug build's checks
       // (r1 is read only by widths with a second plane)
       if (MQ_IN_BOUNDS(r0 + 16 <= st_end && r0b + 16 <= st_end && (b1 == 0 || r1 + 8 <= st_end), p.err))
-        decode32<R>(r0, r0b, r1, v, sub2, subf, ch2, ckm, cs);
+        decode32<R>(r0, r0b, r1, v, sub2, subf, ch2, ckm, cs, epw);
       tc05::st_32x32b_x16(tmem + lane_addr + kASlotCol + s * 32 + h * 16, v);
       tc05::wait_st();
       tc05::fence_before_sync();
@@ -417,9 +451,9 @@ gemm_tc05_kernel(const __grid_constant__ GemmParams p) {
 }
 
 
-template <int R>
+template <int R, bool EP = false>
 cudaError_t launch_gemm_r(const GemmParams& gp, dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = gemm_tc05_kernel<R>;
+  auto kern = gemm_tc05_kernel<R, EP>;
   static std::mutex mu;
   static std::map<int, bool> attr_set;
   int dev = 0;
@@ -445,7 +479,8 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   int b0, b1;
   job_planes(job, b0, b1);
   if (b0 == 0) return cudaErrorInvalidValue;
-  if (job.ep_rows) return cudaErrorNotSupported;  // Extra Precision lists serve the decode path only
+  const bool ep = job.ep_rows != nullptr;
+  if (ep && (job.r == 8 || job.src != kPlanes)) return cudaErrorNotSupported;  // Eq. 8 lists: planes of width <= 6
 
   static thread_local GemmParams gp;
   cudaError_t e = encode_map_2d(&gp.map_x, job.x, uint64_t(M), uint64_t(job.K), 64, kBM, 2, 128);
@@ -464,7 +499,10 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   }
 
   void* ws = nullptr;
-  e = get_workspace(stream, size_t(M) * sizeof(float) + 256, &ws);
+  // Sx, then (Extra Precision) the list's bit plane: N rows of K / 32 words
+  const size_t sx_bytes = (size_t(M) * sizeof(float) + 255) & ~size_t(255);
+  const size_t ep_bytes = ep ? size_t(job.N) * size_t(job.K / 32) * sizeof(uint32_t) : 0;
+  e = get_workspace(stream, sx_bytes + ep_bytes + 256, &ws);
   if (e != cudaSuccess) return e;
   float* sx = static_cast<float*>(ws);
   uint32_t* err = nullptr;
@@ -474,6 +512,14 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   gp.alpha = job.alpha;
   gp.zero = job.zero;
   gp.sx = sx;
+  gp.ep_bits = nullptr;
+  gp.ep_words = static_cast<int>(job.K / 32);
+  if (ep) {
+    uint32_t* bits = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + sx_bytes);
+    e = launch_ep_bits(job.ep_rows, job.ep_cols, job.N, job.K, bits, stream, sm_count());
+    if (e != cudaSuccess) return e;
+    gp.ep_bits = bits;
+  }
   gp.y = job.y;
   gp.err = err;
   gp.wait_ns = wait_limit_ns();
@@ -494,6 +540,15 @@ cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
 
   const dim3 grid(static_cast<unsigned>((job.N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
+  if (ep) {
+    switch (decode_kind(job)) {
+      case 6: return launch_gemm_r<6, true>(gp, grid, smem, stream);
+      case 4: return launch_gemm_r<4, true>(gp, grid, smem, stream);
+      case 3: return launch_gemm_r<3, true>(gp, grid, smem, stream);
+      case 2: return launch_gemm_r<2, true>(gp, grid, smem, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (decode_kind(job)) {
     case 10: return launch_gemm_r<10>(gp, grid, smem, stream);
     case 11: return launch_gemm_r<11>(gp, grid, smem, stream);

@@ -168,6 +168,10 @@ size_t map_table_count();
 // Prefill path (M > 32): tcgen05 GEMM for one linear. Returns
 // cudaErrorNotSupported for shapes it does not serve (nothing launched).
 cudaError_t run_gemm(const LinearJob& job, int M, cudaStream_t stream);
+// An Extra Precision list as a bit plane (N rows of K / 32 words; K % 32 == 0)
+// for the prefill GEMM.
+cudaError_t launch_ep_bits(const int32_t* row_ptr, const uint16_t* cols, int64_t N, int64_t K, uint32_t* bits,
+                           cudaStream_t stream, int sms);
 
 // An NVTX range around every entry point that launches work, so a timeline
 // tool shows each library call (without a tool attached it costs a branch).

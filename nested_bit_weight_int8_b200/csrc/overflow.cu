@@ -138,7 +138,33 @@ uint32_t threshold4(int r) {
   return thr * 0x01010101u;
 }
 
+// The list as a dense bit plane for the prefill GEMM: bit (k % 32) of word
+// n * words + k / 32 is set when position k of row n is listed. One warp per
+// row: it clears the row's words, then sets the listed bits.
+__global__ void __launch_bounds__(kOvfThreads)
+ep_bits_kernel(const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ cols, int64_t N, int words,
+               uint32_t* __restrict__ bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (kOvfThreads / 32);
+  for (int64_t n = (int64_t(blockIdx.x) * kOvfThreads + threadIdx.x) / 32; n < N; n += warps) {
+    uint32_t* row = bits + n * words;
+    for (int w = lane; w < words; w += 32) row[w] = 0u;
+    __syncwarp();
+    const int beg = row_ptr[n], end = row_ptr[n + 1];
+    for (int j = beg + lane; j < end; j += 32) {
+      const int k = cols[j];
+      if (k / 32 < words) atomicOr(row + k / 32, 1u << (k % 32));
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ep_bits(const int32_t* row_ptr, const uint16_t* cols, int64_t N, int64_t K, uint32_t* bits,
+                           cudaStream_t stream, int sms) {
+  ep_bits_kernel<<<ovf_grid(N, sms), kOvfThreads, 0, stream>>>(row_ptr, cols, N, static_cast<int>(K / 32), bits);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ovf_rows(const uint8_t* q, int64_t N, int64_t K, int r, int32_t* row_ptr,
                             cudaStream_t stream, int sms) {

@@ -160,7 +160,7 @@ def test_ep_entry_points_reject():
     assert mq.raw_status("mq_linear_ep", *ok, 8, F, F, F, None) == mq.MQ_ERR_INVALID_ARG   # r = 8
     assert mq.raw_status("mq_linear_ep", *ok, 2, None, F, F, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.raw_status("mq_linear_ep", *ok, 2, F, F + 1, F, None) == mq.MQ_ERR_INVALID_ARG
-    assert mq.raw_status("mq_linear_ep", F, 33, 256, F, F, F, 64, 2, F, F, F, None) == mq.MQ_ERR_UNSUPPORTED
+    assert mq.raw_status("mq_linear_ep", F, 1, 65600, F, F, F, 64, 2, F, F, F, None) == mq.MQ_ERR_UNSUPPORTED
 
 
 def test_debug_build_exports_the_same_entry_points():

@@ -141,3 +141,43 @@ def test_linear_ep_agrees_with_container_eq8():
     x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
     tol = oracle.tolerance(x_vals, oracle.dequant_slice(q, a, z, r, clamp=False))
     assert np.all(np.abs(y1.cpu().numpy() - y2.cpu().numpy()) <= 2 * tol)
+
+
+# Prefill (M > 32): the list goes through a bit plane into the tcgen05 GEMM,
+# whose decode adds one step to every listed code.
+@pytest.mark.parametrize("r", [6, 4, 3, 2])
+@pytest.mark.parametrize("m", [33, 300])
+def test_linear_ep_prefill(r, m):
+    _ep_case(2048, 4096, 60 + r, r, m, 600 + m)
+
+
+@pytest.mark.parametrize("n,k,r,m", [(14336, 4096, 2, 40), (130, 4224, 2, 64), (257, 4128, 4, 70),
+                                     (300, 192, 6, 33), (1000, 384, 3, 257)])
+def test_linear_ep_prefill_shapes(n, k, r, m):
+    # K = 4128 at r = 4 ends halfway through a 64-code stage: the half past K
+    # has no bit-plane word and adds nothing
+    _ep_case(n, k, 70 + n, r, m, 71 + k)
+
+
+def test_linear_ep_prefill_dense_bucket():
+    _ep_case(2048, 4096, 44, 2, 96, 45, frac=0.5)
+
+
+def test_linear_ep_prefill_agrees_with_container_eq8():
+    n, k, r, m = 4096, 4096, 2, 64
+    w = _weights(n, k, 52)
+    q, a, z = oracle.quantize_minmax(w)
+    q_dev = to_dev(q)
+    packed = gpu_pack(q_dev, r)
+    rows, cols, _ = gpu_list(q_dev, n, k, r)
+    x_bits = synth.activations(m, k, 53)
+    x = to_dev(x_bits)
+    y1 = torch.empty((m, n), dtype=torch.float32, device=DEV)
+    y2 = torch.empty((m, n), dtype=torch.float32, device=DEV)
+    mq.linear_ep(x, m, k, packed, to_dev(a), to_dev(z), n, r, rows, cols, y1)
+    mq.linear_container(x, m, k, q_dev, to_dev(a), to_dev(z), n, r, False, y2)
+    torch.cuda.synchronize()
+    x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
+    w8 = oracle.dequant_slice(q, a, z, r, clamp=False)
+    check_linear(y1.cpu().numpy().astype(np.float64), x_vals, w8, "prefill ep, planes + list")
+    check_linear(y2.cpu().numpy().astype(np.float64), x_vals, w8, "prefill ep, container")
