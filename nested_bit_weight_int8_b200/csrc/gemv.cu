@@ -79,12 +79,15 @@ namespace {
 constexpr int kConsumerWarps = 8;
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxStages = 8;
-// Header: barriers and flags from byte 0, a 64-byte zero block ending at
-// byte 1024, then each consumer warp's row scales (alpha and z of its 32
-// rows, 256 bytes a warp) up to byte 3072, where the stages start.
+// Header: barriers and flags from byte 0, each consumer warp's output and
+// Extra Precision pointers (16 bytes a warp) from byte 256, a 64-byte zero
+// block ending at byte 1024, then each consumer warp's row scales (alpha and
+// z of its 32 rows, 256 bytes a warp) up to byte 3072, where the stages start.
 constexpr int kHeaderBytes = 3072;
+constexpr int kPtrsOff = 256;
 constexpr int kScalesOff = 1024;
 static_assert(kScalesOff + kConsumerWarps * 64 * 4 <= kHeaderBytes, "row scales overflow the header");
+static_assert(kPtrsOff + kConsumerWarps * 16 <= kScalesOff - 64, "pointer slots overlap the zero block");
 constexpr int kMaxDynSmem = 227 * 1024;
 constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header and alignment slack
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
@@ -523,15 +526,24 @@ __device__ __forceinline__ void cursor_next(const GemvParams<CAP>& p, Cursor& c)
 // (cp.async, waited for before their first use); rows past N read as zero.
 // The scales do not change during a launch, so the first copy is issued
 // before the wait for the previous grid.
+//
+// Lane 0 also keeps the linear's y and Extra Precision pointers in the
+// warp's slot `ptrs`: read here, at the start of the row block, their load
+// from the kernel parameters (a cold line on every call) is off the flush's
+// path.
 template <int NT, int CAP>
 __device__ __forceinline__ void stage_scales(const GemvParams<CAP>& p, int l, int rb, int warp, int lane,
-                                             float* sc) {
+                                             float* sc, const void** ptrs) {
   const LinDesc& L = p.lin[l];
   const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + lane;
   const bool in = lane < Tiling<NT>::RPW && n < L.N;
   cp_async_4(sc + lane, in ? L.alpha + n : L.alpha, in ? 4u : 0u);
   cp_async_4(sc + 32 + lane, in ? L.zero + n : L.zero, in ? 4u : 0u);
   cp_async_commit();
+  if (lane == 0) {
+    ptrs[0] = L.y;
+    ptrs[1] = L.epc;
+  }
 }
 
 // Epilogue of one row block of this warp's 16 rows: scales the raw sums,
@@ -543,14 +555,19 @@ __device__ __forceinline__ void stage_scales(const GemvParams<CAP>& p, int l, in
 // of the part's units. A row block this CTA owns whole is stored; a shared one
 // is added atomically into y, zeroed first (by the prep kernel, or inside a
 // launch without one).
+//
+// Everything it reads is at hand (the cursor's N, r and kind, the staged
+// scales and pointers): no kernel-parameter load on the flush's path.
 template <int NT, int CAP>
 __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, bool whole, int warp,
-                           int lane, const float (&tot)[Tiling<NT>::TW][NT][4], float sxs, const float* sc) {
+                           int lane, const float (&tot)[Tiling<NT>::TW][NT][4], float sxs, const float* sc,
+                           const void* const* ptrs, int N, int r, int dk, int M) {
   constexpr int TW = Tiling<NT>::TW;
-  const LinDesc& L = p.lin[l];
+  float* const y = static_cast<float*>(const_cast<void*>(ptrs[0]));  // L.y, staged
+  const float* const epc = static_cast<const float*>(ptrs[1]);       // L.epc, staged
   const int g = lane >> 2, t = lane & 3;
-  const float scale = static_cast<float>(1 << (8 - L.r));
-  const int cmax = L.dk == 11 ? (1 << L.r) : (1 << L.r) - 1;
+  const float scale = static_cast<float>(1 << (8 - r));
+  const int cmax = dk == 11 ? (1 << r) : (1 << r) - 1;
   // the row scales, staged in shared memory (stage_scales)
   float av[TW][2], zv[TW][2];
 #pragma unroll
@@ -566,25 +583,25 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int n = rb * Tiling<NT>::RPU + warp * Tiling<NT>::RPW + 16 * T + Tiling<NT>::frag_row(g) + 8 * h;
-      if (n >= L.N) continue;
+      if (n >= N) continue;
       const float a = av[T][h], z = zv[T][h];
       // the same centre code the decode subtracted (make_rowsub)
-      const float c0 = is_i8(L.dk) ? 0.f : static_cast<float>(centre_code(z, L.r, cmax));
+      const float c0 = is_i8(dk) ? 0.f : static_cast<float>(centre_code(z, r, cmax));
       const float A = a * scale, B = a * (z - c0 * scale);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int m = nt * 8 + 2 * t + e;
-          if (m >= p.M) continue;
+          if (m >= M) continue;
           float v = tot[T][nt][2 * h + e];
-          if (is_i8(L.dk)) {
-            if (kc0 == 0 && L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
+          if (is_i8(dk)) {
+            if (kc0 == 0 && epc) v += epc[static_cast<int64_t>(m) * N + n];
             v = A * v - B * sxs;
           } else if (kc0 == 0) {
             // Extra Precision: each listed position adds one code step
-            if (L.epc) v += L.epc[static_cast<int64_t>(m) * L.N + n];
-            const float* P = L.psum + m * kClasses;
+            if (epc) v += epc[static_cast<int64_t>(m) * N + n];
+            const float* P = p.lin[l].psum + m * kClasses;
             float Sx = 0.f;
 #pragma unroll
             for (int i = 0; i < kClasses; ++i) Sx += P[i];
@@ -592,7 +609,7 @@ __device__ void flush_rows(const GemvParams<CAP>& p, int l, int rb, int kc0, boo
           } else {
             v = A * v;
           }
-          float* dst = L.y + static_cast<int64_t>(m) * L.N + n;
+          float* dst = y + static_cast<int64_t>(m) * N + n;
           if (whole) *dst = v;
           else atomicAdd(dst, v);
         }
@@ -1202,10 +1219,11 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
   // This warp's row scales slots; the first segment's copy goes out before
   // the wait for the previous grid (the scales are constant).
   float* sc = reinterpret_cast<float*>(base + kScalesOff) + warp * 64;
+  const void** ptrs = reinterpret_cast<const void**>(base + kPtrsOff) + 2 * warp;
   {
     Cursor c1;
     cursor_init<TL::RPU>(p, u0, c1);
-    stage_scales<NT>(p, c1.l, c1.rb, warp, lane, sc);
+    stage_scales<NT>(p, c1.l, c1.rb, warp, lane, sc, ptrs);
   }
   // Class sums and the zeroed outputs come from the prep kernel; without one
   // (FUSE), the consumers zero the row block this CTA starts inside (the CTA
@@ -1224,6 +1242,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
     named_bar_sync(1, kConsumerWarps * 32);
   }
   const int g = lane >> 2, t = lane & 3;
+  const int M_rows = p.M;
   uint32_t xaddr[NT], xstep[NT];
   const uint32_t zero_addr = static_cast<uint32_t>(zero_block - smem) + t * 16;  // shared offset
 #pragma unroll
@@ -1247,7 +1266,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       // the previous copy has landed (and the flush read it) before the slots are reused
       cp_async_wait_all();
       __syncwarp();
-      stage_scales<NT>(p, c.l, c.rb, warp, lane, sc);
+      stage_scales<NT>(p, c.l, c.rb, warp, lane, sc, ptrs);
     }
     first_seg = false;
     const int seg = min(c.n_kc - c.kc, u1 - u);
@@ -1319,7 +1338,7 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       }
       cp_async_wait_all();  // the row scales (bf16 segments waited already)
       __syncwarp();
-      flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot, sxs, sc);
+      flush_rows<NT>(p, c.l, c.rb, kc0, whole, warp, lane, tot, sxs, sc, ptrs, c.N, c.r, c.dk, M_rows);
     }
     u += seg;
     c.kc += seg;
