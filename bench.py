@@ -266,7 +266,8 @@ def rows_timings(dev, stream):
     quantize (Eq. 1 and Eq. 3's clipped variant), slice-pack (Eq. 6) per
     width, one decode linear per width (M = 1), the decode linear sliced on
     load from the container (Eq. 6 and Eq. 8), Extra Precision from the r = 2
-    planes plus its sparse list, and the prefill GEMM at M = 2048."""
+    planes plus its sparse list, and the prefill GEMM at M = 2048 (from the
+    planes, from the container, and with Extra Precision)."""
     import torch
     import nested_bit_weight_int8_b200 as mq
     n, k = 14336, 4096
@@ -378,7 +379,22 @@ def rows_timings(dev, stream):
             tf = 2 * m * n_p * k_p / us / 1e6
             out[f"prefill_container_{name}_r{r}_{tag}_M{m}"] = {
                 "us": round(us, 2), "TFLOPs": round(tf, 1), "frac_of_bf16_peak": round(tf / bf16_peak, 3)}
-        del q_p, xm, ym
+        # Extra Precision (Eq. 8) at r = 2 from the planes plus the list of
+        # extra-bucket positions (of these Gaussian weights, the top tail)
+        p2 = torch.empty(mq.packed_bytes(n_p, k_p, 2), dtype=torch.uint8, device=dev)
+        mq.slice_pack(q_p, n_p, k_p, 2, p2, stream)
+        rows_p = torch.empty(n_p + 1, dtype=torch.int32, device=dev)
+        mq.ep_overflow_rows(q_p, n_p, k_p, 2, rows_p, stream)
+        torch.cuda.synchronize()
+        nnz_p = int(rows_p[n_p].item())
+        cols_p = torch.empty(max(nnz_p, 8), dtype=torch.int16, device=dev)
+        mq.ep_overflow_cols(q_p, n_p, k_p, 2, rows_p, cols_p, stream)
+        us = timed(lambda: mq.linear_ep(xm, m, k_p, p2, a_p, z_p, n_p, 2, rows_p, cols_p, ym, stream), reps=5)
+        tf = 2 * m * n_p * k_p / us / 1e6
+        out[f"prefill_linear_ep_{name}_r2_M{m}"] = {
+            "us": round(us, 2), "TFLOPs": round(tf, 1), "frac_of_bf16_peak": round(tf / bf16_peak, 3),
+            "extra_bucket_frac": round(nnz_p / (n_p * k_p), 5)}
+        del q_p, xm, ym, p2, rows_p, cols_p
     torch.cuda.synchronize()
     return out
 

@@ -11,16 +11,19 @@
 // an r = 8 unit in the same bytes). A CTA walks its range one row block at a
 // time; a row block it owns whole is stored into y directly, a row block
 // shared with a neighbour is added into y with fp32 atomics, and the prep
-// kernel zeroes exactly those shared row blocks first.
+// kernel zeroes exactly those shared row blocks first (a short integer launch
+// without a prep kernel zeroes them itself, before a grid barrier).
 //
 // CTA = 8 consumer warps + 1 producer warp. The producer stages each unit in
 // shared memory with one 2-D TMA box per plane (cp.async.bulk.tensor; rows
 // past N and bytes past K read as zero) plus one bulk copy of the unit's
-// activation block, signalling an mbarrier. Up to 8 batch rows each consumer
-// warp owns two 16-row tiles (128-byte plane rows in the 128-byte swizzle,
-// 256-row units); above 8 it owns one tile (64-byte rows, 128-row units). It
-// runs mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the weights as the A
-// operand and the batch (n8 tiles) as B.
+// activation block from the prep kernel's layout, or, without a prep kernel,
+// the block computed from x by the producer warp itself; either signals an
+// mbarrier. Up to 8 batch rows each consumer warp owns two 16-row tiles
+// (128-byte plane rows in the 128-byte swizzle, 256-row units); above 8 it
+// owns one tile (64-byte rows, 128-row units). It runs mma.sync m16n8k16
+// (bf16 in, fp32 accumulate) with the weights as the A operand and the batch
+// (n8 tiles) as B.
 //
 // One batch row at r = 8, 4, 2 runs on the integer tensor cores instead
 // (mma.sync m16n8k32, u8 x s8 -> s32): the codes are the A operand as plain

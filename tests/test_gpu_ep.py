@@ -181,3 +181,26 @@ def test_linear_ep_prefill_agrees_with_container_eq8():
     w8 = oracle.dequant_slice(q, a, z, r, clamp=False)
     check_linear(y1.cpu().numpy().astype(np.float64), x_vals, w8, "prefill ep, planes + list")
     check_linear(y2.cpu().numpy().astype(np.float64), x_vals, w8, "prefill ep, container")
+
+
+@pytest.mark.parametrize("r", [4, 2])
+def test_linear_ep_prefill_9b_up_sampled_rows(r):
+    """The 9B-shaped `up` matrix at M = 2048 from the planes plus the list;
+    rows are quantized independently, so the oracle on a row sample is exact."""
+    n, k, m = 14336, 3584, 2048
+    w = _weights(n, k, 80 + r)
+    q, a, z = oracle.quantize_minmax(w)
+    q_dev = to_dev(q)
+    packed = gpu_pack(q_dev, r)
+    rows_l, cols_l, total = gpu_list(q_dev, n, k, r)
+    assert total > 0
+    x_bits = synth.activations(m, k, 90 + r)
+    x_vals = synth.f32_from_bf16_bits(x_bits).astype(np.float64)
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device=DEV)
+    mq.linear_ep(to_dev(x_bits), m, k, packed, to_dev(a), to_dev(z), n, r, rows_l, cols_l, y)
+    mq.device_status()
+    rng = np.random.default_rng(r)
+    rows = np.unique(np.concatenate([rng.choice(n, size=48, replace=False), [0, 127, 128, n - 1]]))
+    y_rows = y.cpu().numpy()[:, rows].astype(np.float64)
+    check_linear(y_rows, x_vals, oracle.dequant_slice(q[rows], a[rows], z[rows], r, clamp=False),
+                 f"prefill ep 9B up r={r} M={m} (sampled rows)")
