@@ -96,6 +96,7 @@ constexpr size_t kStageBudget = 108 * 1024;  // two CTAs per SM with the header 
 constexpr int kMaxCtas = 320;       // persistent grid cap (2 CTAs on each of 148 SMs fit)
 constexpr int kClasses = 8;         // activation classes (k >> 1) & 7
 constexpr int kFuseUnitsPerCta = 8; // integer launches up to this many units per CTA skip the prep kernel
+static_assert(kMaxStages <= kConsumerWarps, "one consumer warp stages each of the first stages' blocks");
 
 // Decode kinds of the planes at one batch row on the integer tensor cores:
 // kDkI8 + r for r = 8, 4, 2. A unit is 256 rows x 128 plane bytes (1024 / r
@@ -1109,6 +1110,11 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       const int pre = min(S, u1 - u0);
       if (lane == 0)
         for (int i = 0; i < pre; ++i) { issue_weights(c, i); cursor_next<TL::RPU>(p, c); }
+      // the first stages' transaction counts are set before any warp arrives
+      // on their barriers: the producer stages unit 0 at once, consumer warp
+      // i the block of unit i for the other first stages (the producer only
+      // signals; the consumers wait)
+      named_bar_arrive(2, kGemvThreads);
       c = pre_c;
       for (int i = 0; i < pre; ++i) cursor_next<TL::RPU>(p, c);
       pdl_wait_primary();
@@ -1126,7 +1132,8 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
           cursor_next<TL::RPU>(p, pc);
         }
       }
-      for (int i = 0; i < pre; ++i) { stage_x(pre_c, i); cursor_next<TL::RPU>(p, pre_c); }
+      stage_x(pre_c, 0);  // unit 0 (pre >= 1 in a CTA with units)
+      for (int i = 0; i < pre; ++i) cursor_next<TL::RPU>(p, pre_c);
       int issued = pre;
       for (int u = u0 + pre; u < u1; ++u, ++issued) {
         const int s = issued % S;
@@ -1243,6 +1250,24 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
     named_bar_sync(1, kConsumerWarps * 32);
     if (threadIdx.x == 0) *s_gen = grid_arrive(p.sync);
     named_bar_sync(1, kConsumerWarps * 32);
+    // Consumer warp i (i >= 1) stages the activation block of the CTA's unit
+    // i into stage i for the first min(stages, units) units, all at once
+    // (the producer, which stages unit 0, would stage them one after
+    // another), and arrives on its full barrier; the producer set the stage's
+    // transaction count before the barrier below.
+    named_bar_sync(2, kGemvThreads);
+    if (warp >= 1 && warp < min(S, u1 - u0)) {
+      Cursor cw;
+      cursor_init<TL::RPU>(p, u0 + warp, cw);
+      const LinDesc& L = p.lin[cw.l];
+      const uint16_t* xr = reinterpret_cast<const uint16_t*>(L.xf);  // the input row itself
+      uint8_t* blk = stages + static_cast<size_t>(warp) * p.stage_bytes + p.off_x;
+      if (cw.dk == kDkI8 + 8) stage_i8_unit<8>(xr, L.K, cw.kc, blk, lane);
+      else if (cw.dk == kDkI8 + 4) stage_i8_unit<4>(xr, L.K, cw.kc, blk, lane);
+      else stage_i8_unit<2>(xr, L.K, cw.kc, blk, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[warp]);
+    }
   }
   const int g = lane >> 2, t = lane & 3;
   const int M_rows = p.M;

@@ -183,6 +183,11 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Arrives at a named barrier without waiting (the threads that wait use
+// named_bar_sync with the same total count).
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 // ---------------------------------------------------------------- MMA
 // D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
