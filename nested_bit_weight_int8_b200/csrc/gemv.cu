@@ -1113,7 +1113,9 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       // the first stages' transaction counts are set before any warp arrives
       // on their barriers: the producer stages unit 0 at once, consumer warp
       // i the block of unit i for the other first stages (the producer only
-      // signals; the consumers wait)
+      // signals; the consumers wait). Named barriers are warp-aligned: the
+      // warp reconverges after lane 0's loop first.
+      __syncwarp();
       named_bar_arrive(2, kGemvThreads);
       c = pre_c;
       for (int i = 0; i < pre; ++i) cursor_next<TL::RPU>(p, c);
@@ -1247,8 +1249,10 @@ gemv_streamk_kernel(const __grid_constant__ GemvParams<CAP> p) {
       const int n = c0c.rb * TL::RPU + static_cast<int>(threadIdx.x);  // one row per consumer thread
       if (n < c0c.N) p.lin[c0c.l].y[n] = 0.f;
     }
+    __syncwarp();  // named barriers are warp-aligned
     named_bar_sync(1, kConsumerWarps * 32);
     if (threadIdx.x == 0) *s_gen = grid_arrive(p.sync);
+    __syncwarp();
     named_bar_sync(1, kConsumerWarps * 32);
     // Consumer warp i (i >= 1) stages the activation block of the CTA's unit
     // i into stage i for the first min(stages, units) units, all at once
