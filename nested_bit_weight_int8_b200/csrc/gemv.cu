@@ -184,18 +184,18 @@ struct GemvParams {
 // kernel parameters are limited to 32764 bytes
 static_assert(sizeof(GemvParams<kGemvMaxLinears>) <= 32764, "decode kernel parameters too large");
 
-// Geometry of one width: plane widths, 8-code activation groups per 16-byte
-// low-plane chunk (W8).
+// Geometry of one width: the high plane's width (b1, 0 for one plane), and
+// the 8-code activation groups per 16-byte low-plane chunk (W8).
 template <int R> struct Geo;
-template <> struct Geo<2> { static constexpr int b0 = 2, b1 = 0, W8 = 8; };
-template <> struct Geo<4> { static constexpr int b0 = 4, b1 = 0, W8 = 4; };
-template <> struct Geo<8> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
-template <> struct Geo<3> { static constexpr int b0 = 2, b1 = 1, W8 = 8; };
-template <> struct Geo<6> { static constexpr int b0 = 4, b1 = 2, W8 = 4; };
+template <> struct Geo<2> { static constexpr int b1 = 0, W8 = 8; };
+template <> struct Geo<4> { static constexpr int b1 = 0, W8 = 4; };
+template <> struct Geo<8> { static constexpr int b1 = 0, W8 = 2; };
+template <> struct Geo<3> { static constexpr int b1 = 1, W8 = 8; };
+template <> struct Geo<6> { static constexpr int b1 = 2, W8 = 4; };
 // The container sliced on load (Eq. 6: kind 10, Eq. 8: kind 11) streams the
 // 8-bit plane.
-template <> struct Geo<10> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
-template <> struct Geo<11> { static constexpr int b0 = 8, b1 = 0, W8 = 2; };
+template <> struct Geo<10> { static constexpr int b1 = 0, W8 = 2; };
+template <> struct Geo<11> { static constexpr int b1 = 0, W8 = 2; };
 
 // Per-linear constants of the slice-on-load decode (both 16-bit halves):
 // h2 the rounding addend 2^(s-1), kmask the code's bits after the shift, mag
