@@ -57,15 +57,19 @@ def test_seven_digits_reconstruct_every_input_exactly(seed):
         assert back * 2.0 ** (E - 48) == float(value)
 
 
-def test_window_is_41_octaves_of_the_top_exponent():
-    # an input whose lowest significant bit lies 48 places below E is still
-    # an integer X; one place more and it is not
-    for top in (-60, 0, 90):
-        m = 0x80  # 8 significant bits: exponent of the lowest bit f = top - 7
-        f = top - 7
-        assert f >= top - 48                    # any input within 41 octaves below
-        low = top - 48                          # the smallest f the digits hold
-        assert (top - low) - 7 == 41
+def test_window_is_where_the_digits_stay_exact():
+    """X = m 2^(f + 48 - E) is an integer for every significand m exactly when
+    f >= E - 48; one place lower an odd m would lose its last bit, which is
+    why such a unit takes the bf16 path. With 8 significant bits, the lowest
+    exact input sits 48 - 7 = 41 octaves below the unit's top octave."""
+    for E in (-60, 0, 90):
+        for m in (1, 3, 0x81, 0xFF):
+            f = E - 48
+            assert (m * 2 ** (f + 48 - E)) == m                 # an integer, held by the digits
+            f = E - 49
+            assert (m * 2.0 ** (f + 48 - E)) % 1 != 0           # odd m: half a unit lost
+        top_of_lowest = (E - 48) + 7
+        assert E - top_of_lowest == 41
 
 
 @pytest.mark.parametrize("r,code_multiple,codes_per_unit", [(8, 1, 128), (4, 16, 256), (2, 64, 512)])
