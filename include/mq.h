@@ -28,9 +28,12 @@
  *    reports MQ_ERR_BOUNDS. The normal build compiles the checks out.
  *  - No C++ exception crosses this interface.
  *  - The library keeps a small per-(device, stream) workspace of device
- *    memory for its own scratch (activation copies, row sums, error word).
- *    It is allocated on first use by a call on that stream; make one call
- *    before capturing such a stream into a CUDA graph. mq_release_workspace()
+ *    memory for its own scratch (activation copies, row sums, the two
+ *    grid-barrier words of short decode calls, error word). It is allocated
+ *    on first use by a call on that stream; make one call before capturing
+ *    such a stream into a CUDA graph. Calls on one stream use its workspace
+ *    in order, so a graph captured on a stream must not run concurrently
+ *    with other calls on that stream's workspace. mq_release_workspace()
  *    frees all of it.
  */
 #ifndef MQ_H_
