@@ -92,12 +92,18 @@ cudaError_t get_workspace(cudaStream_t stream, size_t bytes, void** out, uint32_
     }
     size_t sz = bytes < (1u << 20) ? (1u << 20) : bytes;
     sz = (sz + 4095) & ~size_t(4095);
-    e = cudaMalloc(&w.ptr, sz);
+    void* p = nullptr;
+    e = cudaMalloc(&p, sz);
     if (e != cudaSuccess) return e;
+    // the barrier words start at zero, ahead of any kernel on this stream;
+    // the workspace is kept only once that is enqueued
+    e = cudaMemsetAsync(p, 0, kSyncBytes, stream);
+    if (e != cudaSuccess) {
+      cudaFree(p);
+      return e;
+    }
+    w.ptr = p;
     w.bytes = sz;
-    // the barrier words start at zero, ahead of any kernel on this stream
-    e = cudaMemsetAsync(w.ptr, 0, kSyncBytes, stream);
-    if (e != cudaSuccess) return e;
   }
   *out = static_cast<uint8_t*>(w.ptr) + kSyncBytes;
   if (sync) *sync = static_cast<uint32_t*>(w.ptr);
