@@ -249,3 +249,8 @@ def test_header_is_plain_c_and_links_from_c(tmp_path):
                         "-o", str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_map_table_count_needs_no_device():
+    # a host-side count of the tensor-map tables: none before any stack launch
+    assert mq.debug_map_table_count() == 0
